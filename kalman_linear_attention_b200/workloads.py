@@ -1,0 +1,188 @@
+"""Seeded synthetic inputs for the KLA filter (shapes, distributions, seeds).
+
+This module holds no arithmetic of the filter itself: it only draws the four
+per-token inputs (a, p, phi, b) and the prior (lambda_0, eta_0) of the five
+standard workloads.  Both the CUDA path (tests, bench) and the fp64 oracle read
+their inputs from here, so that they see bit-identical values.
+
+Recipe (fixed, documented in the design notes):
+
+* Each input array k in (a, p, phi, b) has its own stream
+  ``np.random.Generator(np.random.PCG64(SeedSequence(seed).spawn(4)[k]))``.
+* Each stream is drawn in fp64, in C order over [B, T, H, N] (N fastest),
+  in blocks of whole (b, t) rows; block boundaries do not change the values.
+* fp64 draws are rounded to fp32 (numpy cast).  bf16 workloads further round
+  the fp32 values to bf16 (round to nearest even on the bit pattern) and keep
+  them in fp32 arrays, so the values are exactly bf16-representable.
+* lambda_0 = 1 and eta_0 = 0 for every channel, as fp32 [B, H, N].
+
+Distributions ("logU(lo, hi)" = exp(U(ln lo, ln hi)); softplus(x) = ln(1+e^x);
+sigmoid(x) = 1/(1+e^-x); all evaluated in fp64):
+
+* ``base``:  a ~ U(0.5, 1), p ~ logU(1e-3, 1), phi ~ logU(1e-2, 10), b ~ N(0, 1)
+* ``lm``:    a = sigmoid(N(2, 1)), p = softplus(N(-3, 1)), phi = softplus(N(0, 1)),
+             b ~ N(0, 1)
+* ``stiff``: a ~ U(0.99, 1), p ~ logU(1e-6, 1e-3), phi ~ logU(1e-3, 1e3),
+             b ~ N(0, 1)
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass
+from typing import Dict, Iterator, Tuple
+
+import numpy as np
+
+INPUT_NAMES = ("a", "p", "phi", "b")
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    T: int
+    dtype: str          # "f32" or "bf16": the dtype of a, p, phi, b on the device
+    dist: str           # "base", "lm" or "stiff"
+    seed: int
+    decode: bool = False  # True: T sequential one-token decode steps
+    summary: str = ""
+
+    @property
+    def channels(self) -> int:
+        return self.B * self.H * self.N
+
+    @property
+    def token_channels(self) -> int:
+        return self.B * self.T * self.H * self.N
+
+    def with_shape(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": Workload("tiny", 1, 1, 64, 256, "f32", "base", 0,
+                     summary="tiny forward scan, fp32, B=1 H=1 N=64 T=256"),
+    "lm_layer": Workload("lm_layer", 8, 16, 128, 2048, "bf16", "lm", 1,
+                         summary="LM-layer-shaped forward scan, bf16 in / fp32 state, "
+                                 "B=8 H=16 N=128 T=2048"),
+    "long": Workload("long", 1, 32, 128, 65536, "f32", "base", 2,
+                     summary="long-sequence forward scan, fp32, B=1 H=32 N=128 T=65536"),
+    "stiff": Workload("stiff", 256, 8, 64, 128, "f32", "stiff", 3,
+                      summary="stiff state-tracking-shaped scan, fp32, B=256 H=8 N=64 T=128"),
+    "decode": Workload("decode", 256, 32, 128, 1024, "f32", "base", 4, decode=True,
+                       summary="recurrent decode, fp32 resident state, B=256 H=32 N=128, "
+                               "1024 one-token steps"),
+}
+
+# Elements drawn per block; any value gives the same arrays.
+_BLOCK_ELEMS = 1 << 24
+
+
+def _log_uniform(rng: np.random.Generator, lo: float, hi: float, n: int) -> np.ndarray:
+    return np.exp(rng.uniform(np.log(lo), np.log(hi), n))
+
+
+def _softplus(x: np.ndarray) -> np.ndarray:
+    return np.logaddexp(0.0, x)
+
+
+def _sigmoid(x: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _draw(dist: str, name: str, rng: np.random.Generator, n: int) -> np.ndarray:
+    """n fp64 values of input `name` under distribution family `dist`."""
+    if dist == "base":
+        if name == "a":
+            return rng.uniform(0.5, 1.0, n)
+        if name == "p":
+            return _log_uniform(rng, 1e-3, 1.0, n)
+        if name == "phi":
+            return _log_uniform(rng, 1e-2, 10.0, n)
+        return rng.standard_normal(n)
+    if dist == "lm":
+        if name == "a":
+            return _sigmoid(rng.normal(2.0, 1.0, n))
+        if name == "p":
+            return _softplus(rng.normal(-3.0, 1.0, n))
+        if name == "phi":
+            return _softplus(rng.normal(0.0, 1.0, n))
+        return rng.standard_normal(n)
+    if dist == "stiff":
+        if name == "a":
+            return rng.uniform(0.99, 1.0, n)
+        if name == "p":
+            return _log_uniform(rng, 1e-6, 1e-3, n)
+        if name == "phi":
+            return _log_uniform(rng, 1e-3, 1e3, n)
+        return rng.standard_normal(n)
+    raise ValueError(f"unknown distribution family {dist!r}")
+
+
+def round_to_bf16(x32: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest bf16 (ties to even); result stays fp32."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32)
+
+
+def _streams(seed: int):
+    children = np.random.SeedSequence(seed).spawn(len(INPUT_NAMES))
+    return [np.random.Generator(np.random.PCG64(c)) for c in children]
+
+
+def iter_rows(w: Workload, rows_per_block: int | None = None
+              ) -> Iterator[Tuple[int, int, Dict[str, np.ndarray]]]:
+    """Yield (row0, row1, arrays) blocks of the flattened (B*T) row axis.
+
+    Each array in ``arrays`` is fp32 of shape [row1 - row0, H, N]; row r is
+    token t = r % T of batch b = r // T.
+    """
+    HN = w.H * w.N
+    rows = w.B * w.T
+    if rows_per_block is None:
+        rows_per_block = max(1, _BLOCK_ELEMS // max(HN, 1))
+    rngs = _streams(w.seed)
+    r0 = 0
+    while r0 < rows:
+        r1 = min(rows, r0 + rows_per_block)
+        out = {}
+        for name, rng in zip(INPUT_NAMES, rngs):
+            x = _draw(w.dist, name, rng, (r1 - r0) * HN).astype(np.float32)
+            if w.dtype == "bf16":
+                x = round_to_bf16(x)
+            out[name] = x.reshape(r1 - r0, w.H, w.N)
+        yield r0, r1, out
+        r0 = r1
+
+
+def generate(w: Workload) -> Dict[str, np.ndarray]:
+    """All inputs of a workload as fp32 arrays: a, p, phi, b [B, T, H, N];
+    lam0, eta0 [B, H, N]."""
+    HN = w.H * w.N
+    full = {k: np.empty((w.B * w.T, w.H, w.N), dtype=np.float32) for k in INPUT_NAMES}
+    if w.B * w.T * HN:
+        for r0, r1, blk in iter_rows(w):
+            for k in INPUT_NAMES:
+                full[k][r0:r1] = blk[k]
+    out = {k: v.reshape(w.B, w.T, w.H, w.N) for k, v in full.items()}
+    out.update(prior(w))
+    return out
+
+
+def prior(w: Workload) -> Dict[str, np.ndarray]:
+    return {"lam0": np.ones((w.B, w.H, w.N), dtype=np.float32),
+            "eta0": np.zeros((w.B, w.H, w.N), dtype=np.float32)}
+
+
+def channel_sample(w: Workload, count: int, seed: int = 12345) -> np.ndarray:
+    """A sorted, seeded sample of flat channel indices (b*H*N + h*N + n)."""
+    C = w.channels
+    count = min(count, C)
+    rng = np.random.default_rng(seed)
+    idx = rng.choice(C, size=count, replace=False)
+    # always include the first and last channel (tile edges)
+    idx = np.unique(np.concatenate([idx, [0, C - 1]]))
+    return idx

@@ -1,0 +1,135 @@
+"""fp64 CPU oracle for the Kalman Linear Attention filter.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+product path (``kalman_linear_attention_b200``) never imports it, and this
+package never imports the product path: the two share no code.
+
+The arithmetic lives in ``kla_oracle.c`` (plain sequential covariance-form
+Kalman filter, fp64, one channel at a time).  This module only compiles it with
+gcc, loads it with ctypes and converts arrays to contiguous fp64 (an exact
+upcast for fp32 and bf16 inputs).
+
+Pins: every function here is pinned by ``tests/test_oracle.py`` against exact
+rational arithmetic, closed forms (Riccati fixed point, precision sums, the
+no-process-noise affine case, the no-observation covariance recursion) and
+invariants; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "kla_oracle.c")
+LIBRARY = os.path.join(_HERE, "libkla_oracle.so")
+
+CFLAGS = ["-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-std=c11"]
+
+
+def build(source: str = SOURCE, output: str = LIBRARY, force: bool = False) -> str:
+    """Compile ``source`` into a shared library at ``output`` with gcc."""
+    if (not force and os.path.exists(output)
+            and os.path.getmtime(output) >= os.path.getmtime(source)):
+        return output
+    tmp = output + ".tmp"
+    subprocess.run(["gcc", *CFLAGS, "-o", tmp, source, "-lm"], check=True)
+    os.replace(tmp, output)
+    return output
+
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+def _f64(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(x: np.ndarray):
+    return x.ctypes.data_as(_D)
+
+
+@dataclass
+class Oracle:
+    """ctypes handle on one compiled copy of the oracle."""
+
+    lib: ctypes.CDLL
+
+    @classmethod
+    def load(cls, path: str | None = None) -> "Oracle":
+        lib = ctypes.CDLL(path or build())
+        lib.kla_oracle_forward.restype = ctypes.c_int
+        lib.kla_oracle_forward.argtypes = [_D] * 10 + [_I64] * 4 + [ctypes.c_int]
+        lib.kla_oracle_step.restype = ctypes.c_int
+        lib.kla_oracle_step.argtypes = [_D] * 8 + [_I64]
+        lib.kla_oracle_max_threads.restype = ctypes.c_int
+        lib.kla_oracle_max_threads.argtypes = []
+        return cls(lib)
+
+    def max_threads(self) -> int:
+        return int(self.lib.kla_oracle_max_threads())
+
+    def forward(self, a, p, phi, b, lam0, eta0, threads: int = 1):
+        """Filter every channel of [B, T, H, N] inputs from the [B, H, N] prior.
+
+        Returns a dict with fp64 arrays ``lam``, ``eta``, ``mu``, ``var`` of
+        shape [B, T, H, N].
+        """
+        a, p, phi, b = (_f64(x) for x in (a, p, phi, b))
+        if a.ndim != 4 or not (a.shape == p.shape == phi.shape == b.shape):
+            raise ValueError("a, p, phi, b must share one [B, T, H, N] shape")
+        B, T, H, N = a.shape
+        lam0 = _f64(np.broadcast_to(np.asarray(lam0, dtype=np.float64), (B, H, N)))
+        eta0 = _f64(np.broadcast_to(np.asarray(eta0, dtype=np.float64), (B, H, N)))
+        out = {k: np.empty((B, T, H, N), dtype=np.float64) for k in ("lam", "eta", "mu", "var")}
+        rc = self.lib.kla_oracle_forward(
+            _ptr(a), _ptr(p), _ptr(phi), _ptr(b), _ptr(lam0), _ptr(eta0),
+            _ptr(out["lam"]), _ptr(out["eta"]), _ptr(out["mu"]), _ptr(out["var"]),
+            B, T, H, N, int(threads))
+        if rc != 0:
+            raise ValueError(f"kla_oracle_forward failed ({rc})")
+        return out
+
+    def step(self, a, p, phi, b, lam_state, eta_state):
+        """One decode token for every channel; returns the new state and outputs.
+
+        Inputs are arrays of one common shape; the state arrays are not
+        modified (copies are advanced and returned).
+        """
+        a, p, phi, b = (_f64(x) for x in (a, p, phi, b))
+        shape = a.shape
+        lam = _f64(lam_state).copy()
+        eta = _f64(eta_state).copy()
+        if not (p.shape == phi.shape == b.shape == lam.shape == eta.shape == shape):
+            raise ValueError("step inputs and state must share one shape")
+        mu = np.empty(shape, dtype=np.float64)
+        var = np.empty(shape, dtype=np.float64)
+        rc = self.lib.kla_oracle_step(_ptr(a), _ptr(p), _ptr(phi), _ptr(b),
+                                      _ptr(lam), _ptr(eta), _ptr(mu), _ptr(var), a.size)
+        if rc != 0:
+            raise ValueError(f"kla_oracle_step failed ({rc})")
+        return {"lam": lam, "eta": eta, "mu": mu, "var": var}
+
+
+_DEFAULT: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``kla_oracle.c`` in this directory."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = Oracle.load()
+    return _DEFAULT
+
+
+def forward(a, p, phi, b, lam0, eta0, threads: int = 1):
+    return default().forward(a, p, phi, b, lam0, eta0, threads=threads)
+
+
+def step(a, p, phi, b, lam_state, eta_state):
+    return default().step(a, p, phi, b, lam_state, eta_state)

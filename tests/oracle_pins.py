@@ -1,0 +1,344 @@
+"""Pins that tie the fp64 oracle to facts other than its own code.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` handle and raises
+``AssertionError`` when the oracle disagrees with the fact it checks.  The facts
+come from the pages' definitions and from mathematics, never from the oracle:
+
+* exact rational arithmetic (Python ``fractions``) of the Moebius precision map
+  M_t = [[1 + p phi, a^2 phi], [p, a^2]] and of the precision-ratio gate
+  f_t = a_t / (a_t^2 + p_t lambda_{t-1}) -- the matrix form of the KLA review
+  ("What carries the argument", and its reference [13] on linear-fractional
+  maps) -- against the oracle's covariance-form filter;
+* the Riccati fixed point of constant parameters, via ``numpy.roots``;
+* special cases with textbook closed forms: the plain precision sum and the
+  precision-weighted average of observations (a = 1, p = 0), the affine case
+  without process noise (p = 0, "c = 0 gives az + b" in reference [13]), the
+  no-observation case (phi = 0: the update leaves the prior unchanged, primer
+  section 5.1) with its geometric-series variance;
+* identities of the map: f_t^2 = d lambda_t / d lambda_{t-1}, and the gate
+  product over a span equals prod(a) / (C lambda_s + D) from the matrix product;
+* invariants: lambda_t > 0, lambda_t - phi_t > 0, var * lambda = 1, mu * lambda = eta.
+
+The same functions run against deliberately broken copies of the oracle in
+``test_oracle_mutants.py``; each broken copy must fail at least one pin.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction as Fr
+
+import numpy as np
+
+from kalman_linear_attention_b200 import workloads as wl
+
+
+# ---------------------------------------------------------------- helpers
+def _rel_close(got, ref, rtol, what):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} vs {ref.shape}"
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    bound = rtol * np.abs(ref)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: max rel err {np.max(err / np.maximum(np.abs(ref), 1e-300)):.3e}"
+                           f" > {rtol:g}")
+
+
+def _scaled_close(got, ref, rtol, what, axis=1):
+    """|got - ref| <= rtol (|ref| + rms(ref along the time axis))."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} vs {ref.shape}"
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    rms = np.sqrt(np.mean(ref * ref, axis=axis, keepdims=True)) if ref.ndim > 1 else \
+        np.sqrt(np.mean(ref * ref))
+    bound = rtol * (np.abs(ref) + rms)
+    err = np.abs(got - ref)
+    assert not (err > bound).any(), f"{what}: max scaled err {np.max(err / (np.abs(ref) + rms)):.3e}"
+
+
+def _as4(x):
+    """[T] -> [1, T, 1, 1]"""
+    return np.asarray(x, dtype=np.float64).reshape(1, -1, 1, 1)
+
+
+# ---------------------------------------------------- exact rational reference
+def _random_fraction(rng, lo, hi, den_max):
+    return Fr(int(rng.integers(lo, hi + 1)), int(rng.integers(1, den_max + 1)))
+
+
+def exact_moebius_filter(a, p, phi, b, lam0, eta0):
+    """Exact rationals: lambda_t from the explicit Moebius matrix product
+    M_t ... M_1 applied to lambda_0, eta_t from the gated affine recursion."""
+    T = len(a)
+    # running product P = M_t ... M_1 as a 2x2 of Fractions
+    A, B_, C, D = Fr(1), Fr(0), Fr(0), Fr(1)
+    lam_prev, eta = lam0, eta0
+    lam_out, eta_out = [], []
+    for t in range(T):
+        m11, m12 = 1 + p[t] * phi[t], a[t] * a[t] * phi[t]
+        m21, m22 = p[t], a[t] * a[t]
+        A, B_, C, D = (m11 * A + m12 * C, m11 * B_ + m12 * D,
+                       m21 * A + m22 * C, m21 * B_ + m22 * D)
+        lam_t = (A * lam0 + B_) / (C * lam0 + D)
+        f_t = a[t] / (a[t] * a[t] + p[t] * lam_prev)
+        eta = f_t * eta + b[t]
+        lam_out.append(lam_t)
+        eta_out.append(eta)
+        lam_prev = lam_t
+    return lam_out, eta_out
+
+
+def exact_homogeneous_filter(a, p, phi, b, lam0, eta0):
+    """Exact rationals: one product of 3x3 block-lower-triangular matrices
+    G_t = [[1+p phi, a^2 phi, 0], [p, a^2, 0], [b p, b a^2, a]] applied to
+    (lambda_0, 1, eta_0); lambda_t = n_t / d_t and eta_t = h_t / d_t."""
+    n, d, h = lam0, Fr(1), eta0
+    lam_out, eta_out = [], []
+    for t in range(len(a)):
+        a2 = a[t] * a[t]
+        n, d, h = ((1 + p[t] * phi[t]) * n + a2 * phi[t] * d,
+                   p[t] * n + a2 * d,
+                   b[t] * p[t] * n + b[t] * a2 * d + a[t] * h)
+        lam_out.append(n / d)
+        eta_out.append(h / d)
+    return lam_out, eta_out
+
+
+def random_rational_problem(seed, B=2, T=10, H=1, N=3, allow_negative_a=True):
+    rng = np.random.default_rng(seed)
+    shape = (B, T, H, N)
+    fr = {}
+    fr["a"] = np.empty(shape, dtype=object)
+    fr["p"] = np.empty(shape, dtype=object)
+    fr["phi"] = np.empty(shape, dtype=object)
+    fr["b"] = np.empty(shape, dtype=object)
+    for idx in np.ndindex(shape):
+        a = _random_fraction(rng, 1, 9, 8)
+        if allow_negative_a and rng.random() < 0.25:
+            a = -a
+        fr["a"][idx] = a
+        fr["p"][idx] = _random_fraction(rng, 0, 6, 8)
+        fr["phi"][idx] = _random_fraction(rng, 0, 6, 8)
+        fr["b"][idx] = _random_fraction(rng, -6, 6, 8)
+    fr["lam0"] = np.empty((B, H, N), dtype=object)
+    fr["eta0"] = np.empty((B, H, N), dtype=object)
+    for idx in np.ndindex((B, H, N)):
+        fr["lam0"][idx] = _random_fraction(rng, 1, 6, 4)
+        fr["eta0"][idx] = _random_fraction(rng, -4, 4, 4)
+    return fr
+
+
+def exact_solution(fr, method=exact_moebius_filter):
+    B, T, H, N = fr["a"].shape
+    lam = np.empty((B, T, H, N), dtype=object)
+    eta = np.empty((B, T, H, N), dtype=object)
+    for bi in range(B):
+        for h in range(H):
+            for n in range(N):
+                sl = (bi, slice(None), h, n)
+                l, e = method(list(fr["a"][sl]), list(fr["p"][sl]), list(fr["phi"][sl]),
+                              list(fr["b"][sl]), fr["lam0"][bi, h, n], fr["eta0"][bi, h, n])
+                lam[sl] = l
+                eta[sl] = e
+    return lam, eta
+
+
+def _to_f64(obj_arr):
+    return np.vectorize(float, otypes=[np.float64])(obj_arr)
+
+
+# ------------------------------------------------------------------- pins
+def pin_exact_rational(orc, seeds=(1, 2, 3)):
+    """fp64 oracle == exact Moebius/affine solution to ~1e-13 (B=2 catches
+    batch-stride mistakes, N=3 and per-channel priors catch channel mix-ups,
+    negative a catches a^2 vs a in the gate)."""
+    for seed in seeds:
+        fr = random_rational_problem(seed)
+        lam_x, eta_x = exact_solution(fr)
+        f64 = {k: _to_f64(v) for k, v in fr.items()}
+        out = orc.forward(f64["a"], f64["p"], f64["phi"], f64["b"], f64["lam0"], f64["eta0"])
+        lam_r = _to_f64(lam_x)
+        eta_r = _to_f64(eta_x)
+        mu_r = _to_f64(eta_x / lam_x)
+        var_r = _to_f64(1 / lam_x)
+        _rel_close(out["lam"], lam_r, 1e-13, f"lambda (seed {seed})")
+        _rel_close(out["var"], var_r, 1e-13, f"var (seed {seed})")
+        _scaled_close(out["eta"], eta_r, 1e-13, f"eta (seed {seed})")
+        _scaled_close(out["mu"], mu_r, 1e-13, f"mu (seed {seed})")
+
+
+def pin_exact_rational_step(orc, seed=7):
+    """The one-token decode step, iterated, equals the exact solution too."""
+    fr = random_rational_problem(seed, B=1, T=8, H=2, N=2)
+    lam_x, eta_x = exact_solution(fr)
+    f64 = {k: _to_f64(v) for k, v in fr.items()}
+    lam, eta = f64["lam0"][0].copy(), f64["eta0"][0].copy()
+    for t in range(f64["a"].shape[1]):
+        o = orc.step(f64["a"][0, t], f64["p"][0, t], f64["phi"][0, t], f64["b"][0, t], lam, eta)
+        lam, eta = o["lam"], o["eta"]
+        _rel_close(lam, _to_f64(lam_x[0, t]), 1e-13, f"step lambda t={t}")
+        _scaled_close(eta.ravel(), _to_f64(eta_x[0, t]).ravel(), 1e-13, f"step eta t={t}")
+        _rel_close(o["var"], _to_f64(1 / lam_x[0, t]), 1e-13, f"step var t={t}")
+        _scaled_close(o["mu"].ravel(), _to_f64(eta_x[0, t] / lam_x[0, t]).ravel(), 1e-13,
+                      f"step mu t={t}")
+
+
+def riccati_fixed_point(a, p, phi):
+    """Positive root of p lam^2 + (a^2 - 1 - p phi) lam - a^2 phi = 0 (numpy.roots)."""
+    roots = np.roots([p, a * a - 1.0 - p * phi, -a * a * phi])
+    pos = [r.real for r in roots if abs(r.imag) < 1e-12 and r.real > 0]
+    assert len(pos) == 1
+    return pos[0]
+
+
+def pin_riccati(orc):
+    """Constant (a, p, phi, b) converge to the Riccati fixed point lambda* and
+    to eta* = b / (1 - f*), f* = a / (a^2 + p lambda*)."""
+    # worked value: a = 0.75, p = 0.03, phi = 0.3
+    lam_star = riccati_fixed_point(0.75, 0.03, 0.3)
+    assert abs(lam_star - 15.2521341800603) < 1e-9
+    f_star = 0.75 / (0.75 ** 2 + 0.03 * lam_star)
+    assert abs(f_star - 0.73524796613) < 1e-9
+    rng = np.random.default_rng(11)
+    cases = [(0.75, 0.03, 0.3, 0.4), (1.0, 0.01, 0.5, -1.0), (0.5, 1.0, 10.0, 2.0),
+             (-0.9, 0.2, 0.05, 1.5)]
+    for _ in range(6):
+        cases.append((rng.uniform(0.5, 1.0), float(np.exp(rng.uniform(np.log(1e-3), 0))),
+                      float(np.exp(rng.uniform(np.log(1e-2), np.log(10)))), rng.standard_normal()))
+    T = 6000
+    for a, p, phi, b in cases:
+        lam_s = riccati_fixed_point(a, p, phi)
+        f_s = a / (a * a + p * lam_s)
+        eta_s = b / (1.0 - f_s)
+        out = orc.forward(_as4(np.full(T, a)), _as4(np.full(T, p)), _as4(np.full(T, phi)),
+                          _as4(np.full(T, b)), [[[2.0]]], [[[0.5]]])
+        _rel_close(out["lam"][0, -1, 0, 0], lam_s, 1e-11, f"lambda* a={a} p={p} phi={phi}")
+        assert abs(out["eta"][0, -1, 0, 0] - eta_s) <= 1e-10 * (abs(eta_s) + 1), \
+            f"eta* a={a} p={p} phi={phi}: {out['eta'][0, -1, 0, 0]} vs {eta_s}"
+        _rel_close(out["mu"][0, -1, 0, 0], eta_s / lam_s, 1e-10, "mu*")
+
+
+def pin_precision_sum(orc):
+    """a = 1, p = 0: lambda_t = lambda_0 + sum phi, eta_t = eta_0 + sum b, and
+    mu_t is the precision-weighted average of the observations y_s = b_s/phi_s
+    and the prior mean (numpy.average)."""
+    rng = np.random.default_rng(5)
+    T = 300
+    phi = np.exp(rng.uniform(np.log(1e-2), np.log(10), T))
+    y = rng.standard_normal(T) * 3 + 1
+    b = phi * y
+    lam0, eta0 = 2.5, -1.25
+    out = orc.forward(_as4(np.ones(T)), _as4(np.zeros(T)), _as4(phi), _as4(b),
+                      [[[lam0]]], [[[eta0]]])
+    lam_ref = np.array([lam0 + math.fsum(phi[:t + 1]) for t in range(T)])
+    eta_ref = np.array([eta0 + math.fsum(b[:t + 1]) for t in range(T)])
+    _rel_close(out["lam"][0, :, 0, 0], lam_ref, 1e-13, "precision sum")
+    _scaled_close(out["eta"][0, :, 0, 0], eta_ref, 1e-13, "information sum")
+    mu0 = eta0 / lam0
+    for t in (0, 1, 17, T - 1):
+        ref = np.average(np.concatenate([[mu0], y[:t + 1]]),
+                         weights=np.concatenate([[lam0], phi[:t + 1]]))
+        got = out["mu"][0, t, 0, 0]
+        assert abs(got - ref) <= 1e-12 * (abs(ref) + 1), f"weighted mean t={t}: {got} vs {ref}"
+
+
+def pin_no_process_noise(orc):
+    """p = 0 (affine Moebius case): brute-force sums of products
+    lambda_t = lambda_0 prod a^-2 + sum_s phi_s prod_{j>s} a_j^-2 and
+    eta_t = eta_0 prod a^-1 + sum_s b_s prod_{j>s} a_j^-1."""
+    rng = np.random.default_rng(9)
+    T = 40
+    a = rng.uniform(0.8, 1.2, T) * np.where(rng.random(T) < 0.3, -1.0, 1.0)
+    phi = rng.uniform(0.0, 2.0, T)
+    b = rng.standard_normal(T)
+    lam0, eta0 = 0.7, 0.3
+    out = orc.forward(_as4(a), _as4(np.zeros(T)), _as4(phi), _as4(b), [[[lam0]]], [[[eta0]]])
+    for t in range(T):
+        lam_ref = lam0 * np.prod(a[:t + 1] ** -2.0)
+        eta_ref = eta0 * np.prod(1.0 / a[:t + 1])
+        for s in range(t + 1):
+            lam_ref += phi[s] * np.prod(a[s + 1:t + 1] ** -2.0)
+            eta_ref += b[s] * np.prod(1.0 / a[s + 1:t + 1])
+        _rel_close(out["lam"][0, t, 0, 0], lam_ref, 1e-12, f"p=0 lambda t={t}")
+        assert abs(out["eta"][0, t, 0, 0] - eta_ref) <= 1e-12 * (abs(eta_ref) + 1), f"p=0 eta t={t}"
+
+
+def pin_no_observation(orc):
+    """phi = 0, b = 0 (missing observations): the update leaves the prior
+    unchanged, so with constant a, p the variance is the geometric series
+    P_t = a^(2t) P_0 + p (1 - a^(2t)) / (1 - a^2) and mu_t = a^t mu_0."""
+    T = 200
+    for a, p in ((0.9, 0.05), (1.1, 0.02), (-0.95, 0.3)):
+        lam0, eta0 = 4.0, 2.0
+        out = orc.forward(_as4(np.full(T, a)), _as4(np.full(T, p)), _as4(np.zeros(T)),
+                          _as4(np.zeros(T)), [[[lam0]]], [[[eta0]]])
+        t = np.arange(1, T + 1)
+        P_ref = a ** (2 * t) / lam0 + p * (1 - a ** (2 * t)) / (1 - a * a)
+        _rel_close(out["var"][0, :, 0, 0], P_ref, 1e-12, f"no-obs variance a={a}")
+        mu_ref = a ** t * (eta0 / lam0)
+        _rel_close(out["mu"][0, :, 0, 0], mu_ref, 1e-12, f"no-obs mean a={a}")
+
+
+def pin_gate_derivative(orc):
+    """f_t^2 = d lambda_t / d lambda_{t-1}: the gate measured on the mean path
+    (b = 0, eta_0 = 1 gives eta_1 = f_1) against a central finite difference of
+    the precision path."""
+    rng = np.random.default_rng(21)
+    for _ in range(20):
+        a = rng.uniform(0.5, 1.0) * (1 if rng.random() < 0.7 else -1)
+        p = float(np.exp(rng.uniform(np.log(1e-3), 0)))
+        phi = float(np.exp(rng.uniform(np.log(1e-2), np.log(10))))
+        lam0 = float(np.exp(rng.uniform(-1, 3)))
+        one = lambda l0, e0, bb: orc.forward(_as4([a]), _as4([p]), _as4([phi]), _as4([bb]),
+                                              [[[l0]]], [[[e0]]])
+        f1 = one(lam0, 1.0, 0.0)["eta"][0, 0, 0, 0]
+        h = 1e-5 * lam0
+        d = (one(lam0 + h, 0.0, 0.0)["lam"][0, 0, 0, 0] -
+             one(lam0 - h, 0.0, 0.0)["lam"][0, 0, 0, 0]) / (2 * h)
+        assert abs(f1 * f1 - d) <= 1e-6 * abs(d), f"f^2={f1 * f1} vs dlam={d}"
+        assert np.sign(f1) == np.sign(a), "gate sign must follow a"
+
+
+def pin_gate_product(orc):
+    """Over a span s..t the product of gates equals prod(a) / (C lambda_s + D),
+    [[A, B], [C, D]] = M_t ... M_{s+1} (numpy matrix products of the pages'
+    M_t).  The gate product is read off the mean path with b = 0, eta_s = 1."""
+    rng = np.random.default_rng(33)
+    w = wl.WORKLOADS["tiny"]
+    for span in (1, 5, 24):
+        a = rng.uniform(0.5, 1.0, span)
+        p = np.exp(rng.uniform(np.log(1e-3), 0, span))
+        phi = np.exp(rng.uniform(np.log(1e-2), np.log(10), span))
+        lam_s = 1.7
+        out = orc.forward(_as4(a), _as4(p), _as4(phi), _as4(np.zeros(span)), [[[lam_s]]], [[[1.0]]])
+        prod = np.eye(2)
+        for t in range(span):
+            M = np.array([[1 + p[t] * phi[t], a[t] ** 2 * phi[t]], [p[t], a[t] ** 2]])
+            prod = M @ prod
+            ref = np.prod(a[:t + 1]) / (prod[1, 0] * lam_s + prod[1, 1])
+            got = out["eta"][0, t, 0, 0]
+            assert abs(got - ref) <= 1e-12 * abs(ref), f"gate product span {t + 1}: {got} vs {ref}"
+            lam_ref = (prod[0, 0] * lam_s + prod[0, 1]) / (prod[1, 0] * lam_s + prod[1, 1])
+            _rel_close(out["lam"][0, t, 0, 0], lam_ref, 1e-12, "Moebius product")
+    del w
+
+
+def pin_invariants(orc):
+    """On every workload's distribution family: lambda_t > 0, the prior
+    precision lambda_t - phi_t > 0 ("update never makes things worse"),
+    var * lambda = 1 and mu * lambda = eta."""
+    for name in ("tiny", "lm_layer", "stiff"):
+        w = wl.WORKLOADS[name].with_shape(B=2, T=64, H=2, N=8)
+        x = wl.generate(w)
+        out = orc.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+        assert np.all(out["lam"] > 0), name
+        assert np.all(out["lam"] - x["phi"] > 0), name
+        _rel_close(out["var"] * out["lam"], np.ones_like(out["lam"]), 1e-14, f"{name} var*lam")
+        _scaled_close(out["mu"] * out["lam"], out["eta"], 1e-14, f"{name} mu*lam")
+
+
+ALL_PINS = [pin_exact_rational, pin_exact_rational_step, pin_riccati, pin_precision_sum,
+            pin_no_process_noise, pin_no_observation, pin_gate_derivative, pin_gate_product,
+            pin_invariants]

@@ -1,0 +1,56 @@
+"""The fp64 oracle against its pins (closed forms, exact rationals, invariants)."""
+import numpy as np
+import pytest
+
+import oracle
+import oracle_pins as pins
+from kalman_linear_attention_b200 import workloads as wl
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.default()
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(orc, pin):
+    pin(orc)
+
+
+def test_exact_forms_agree():
+    """The Moebius/affine form and the 3x3 homogeneous form are the same exact
+    rational recursion (the identity the CUDA path's chunk aggregates rely on)."""
+    for seed in (1, 2):
+        fr = pins.random_rational_problem(seed, B=1, T=9, H=1, N=2)
+        l1, e1 = pins.exact_solution(fr, pins.exact_moebius_filter)
+        l2, e2 = pins.exact_solution(fr, pins.exact_homogeneous_filter)
+        assert (l1 == l2).all() and (e1 == e2).all()
+
+
+def test_step_iterates_to_forward(orc):
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=50, H=2, N=4)
+    x = wl.generate(w)
+    out = orc.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    lam, eta = x["lam0"].astype(np.float64), x["eta0"].astype(np.float64)
+    for t in range(w.T):
+        o = orc.step(x["a"][:, t], x["p"][:, t], x["phi"][:, t], x["b"][:, t], lam, eta)
+        lam, eta = o["lam"], o["eta"]
+        for k in ("lam", "eta", "mu", "var"):
+            assert np.array_equal(o[k], out[k][:, t]), (k, t)
+
+
+def test_threads_do_not_change_results(orc):
+    w = wl.WORKLOADS["stiff"].with_shape(B=4, T=40)
+    x = wl.generate(w)
+    one = orc.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], threads=1)
+    many = orc.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], threads=4)
+    for k in one:
+        assert np.array_equal(one[k], many[k])
+
+
+def test_empty_and_bad_shapes(orc):
+    z = np.zeros((1, 0, 1, 4))
+    out = orc.forward(z, z, z, z, np.ones((1, 1, 4)), np.zeros((1, 1, 4)))
+    assert out["lam"].shape == (1, 0, 1, 4)
+    with pytest.raises(ValueError):
+        orc.forward(np.zeros((1, 2, 1, 4)), z, z, z, 1.0, 0.0)

@@ -1,0 +1,55 @@
+"""Plant one plausible mistake at a time in a copy of the oracle (on the CPU)
+and check that the pin suite rejects every broken copy."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins as pins
+
+MUTANTS = {
+    "dropped process noise": ("a * a * P_prev + p;", "a * a * P_prev;"),
+    "a instead of a^2 in predict": ("a * a * P_prev + p;", "a * P_prev + p;"),
+    "mean not propagated by a": ("const double m_pred = a * m_prev;",
+                                 "const double m_pred = m_prev;"),
+    "evidence precision subtracted": ("*lam_out = 1.0 / P_pred + phi;",
+                                      "*lam_out = 1.0 / P_pred - phi;"),
+    "prior information inverted": ("*eta_out = m_pred / P_pred + b;",
+                                   "*eta_out = m_pred * P_pred + b;"),
+    "token information subtracted": ("*eta_out = m_pred / P_pred + b;",
+                                     "*eta_out = m_pred / P_pred - b;"),
+    "mu = eta * lambda": ("mu[i] = eta_t / lam_t;", "mu[i] = eta_t * lam_t;"),
+    "var = lambda": ("var[i] = 1.0 / lam_t;", "var[i] = lam_t;"),
+    "prior variance = lambda_0": ("double P = 1.0 / lam0;", "double P = lam0;"),
+    "prior mean = eta_0": ("double m = eta0 / lam0;", "double m = eta0;"),
+    "carried mean = eta": ("        m = eta_t / lam_t;", "        m = eta_t;"),
+    "carried variance = prior variance": ("        P = 1.0 / lam_t;",
+                                          "        P = 1.0 / (lam_t - phi[i]);"),
+    "p and phi transposed": ("kf_token(a[i], p[i], phi[i], b[i],",
+                             "kf_token(a[i], phi[i], p[i], b[i],"),
+    "wrong batch stride": ("const int64_t base = bi * T * HN + hn;",
+                           "const int64_t base = bi * HN + hn;"),
+    "prior of channel 0 for all": ("lam0[ch], eta0[ch],", "lam0[0], eta0[0],"),
+    "decode step: state read as variance": ("const double P = 1.0 / lam_state[ch];",
+                                            "const double P = lam_state[ch];"),
+    "decode step: eta not written": ("        eta_state[ch] = eta_t;", "        (void)eta_t;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    with open(oracle.SOURCE) as f:
+        src = f.read()
+    assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.build(str(path), str(tmp_path / "libmutant.so"), force=True)
+    orc = oracle.Oracle.load(os.path.abspath(lib))
+    failures = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError, ZeroDivisionError) as e:
+            failures.append((pin.__name__, str(e)[:80]))
+    assert failures, f"no pin caught mutant {name!r}"
