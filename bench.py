@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the KLA filter scan on B200 (one JSON line on rank 0).
+
+A step is one kla_scan_forward call (load, Moebius + affine chunk scan,
+cross-chunk carry, emit lambda / eta / mu / var) over the long-sequence
+workload (B=1, H=32, N=128, T=65536, fp32): 268.4 M token-channels per GPU,
+8.59 GB of algorithmic HBM traffic.  The same line also reports the recurrent
+decode step (B=256, H=32, N=128, fp32 resident state; 1024 tokens replayed
+from a CUDA graph).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank filters its own
+independent channels (a different seed per rank), so work per GPU is fixed
+("weak" scaling) and no collective touches the data path: the only
+collectives are the barrier and the max-over-ranks of the timings.
+
+``--impl reference`` times the fp64 CPU oracle (the method's plain sequential
+definition) on the host cores, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from kalman_linear_attention_b200 import workloads as wl  # noqa: E402
+
+METRIC = "scan throughput (token-channels/s) and achieved HBM GB/s vs B200 peak, 1 GPU"
+UNIT = "token-channels/s"
+FALLBACK_HBM_GBS = 6650.0
+CSRC = os.path.join(ROOT, "kalman_linear_attention_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+
+
+# --------------------------------------------------------------- host helpers
+def algorithmic_bytes_per_tc(w: wl.Workload) -> int:
+    """Bytes the method must move per token-channel: read a, p, phi, b once,
+    write lambda, eta, mu, var (fp32) once."""
+    return (2 if w.dtype == "bf16" else 4) * 4 + 4 * 4
+
+
+def decode_bytes_per_channel(w: wl.Workload) -> int:
+    """Per decode token and channel: inputs, state read, state write, mu and var."""
+    return (2 if w.dtype == "bf16" else 4) * 4 + 8 + 8 + 8
+
+
+def rank_workload(w: wl.Workload, rank: int) -> wl.Workload:
+    """Each rank filters its own independent channels: same shape, own seed."""
+    return w if rank == 0 else w.with_shape(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, dist_mod=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist_mod is None or not dist_mod.is_initialized() or dist_mod.get_world_size() == 1:
+        return float(x)
+    import torch
+    backend = dist_mod.get_backend()
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only if it was
+    taken on the kernel sources as they are now."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_sha") != kernel_source_hash():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        # under load: samples drawing more than the idle baseline
+        loaded = [s for s, pw in zip(sm, power) if pw is not None and pw > 0.5 * max(power)] if power else sm
+        return {"sm_mhz": statistics.median(loaded or sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------- our arm
+def inputs_to_device(w: wl.Workload, device, keep_host: bool):
+    """Generated inputs, streamed block by block into device tensors [B, T, H, N];
+    optionally also kept as pinned host tensors (for the end-to-end leg)."""
+    import torch
+    B, T, H, N = w.B, w.T, w.H, w.N
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = {k: torch.empty((B, T, H, N), dtype=dt, device=device) for k in wl.INPUT_NAMES}
+    host = {k: torch.empty((B, T, H, N), dtype=dt, pin_memory=True) for k in wl.INPUT_NAMES} \
+        if keep_host else None
+    HN = H * N
+    for r0, r1, blk in wl.iter_rows(w):
+        for k in wl.INPUT_NAMES:
+            x = torch.from_numpy(blk[k].reshape(r1 - r0, HN)).to(dt)
+            dev[k].view(B * T, HN)[r0:r1].copy_(x)
+            if host is not None:
+                host[k].view(B * T, HN)[r0:r1].copy_(x)
+    pri = wl.prior(w)
+    dev["lam0"] = torch.from_numpy(pri["lam0"]).to(device)
+    dev["eta0"] = torch.from_numpy(pri["eta0"]).to(device)
+    if host is not None:
+        host["lam0"] = torch.from_numpy(pri["lam0"]).pin_memory()
+        host["eta0"] = torch.from_numpy(pri["eta0"]).pin_memory()
+    return dev, host
+
+
+def time_forward(kla, w, dev, steps: int, warmup: int, dist_mod):
+    import torch
+    B, T, H, N = w.B, w.T, w.H, w.N
+    outs = [torch.empty((B, T, H, N), dtype=torch.float32, device=dev["a"].device) for _ in range(4)]
+    ws = kla.new_workspace(B, T, H, N, dev["a"].dtype, dev["a"].device)
+    stream = torch.cuda.current_stream()
+    args = (dev["a"], dev["p"], dev["phi"], dev["b"], dev["lam0"], dev["eta0"])
+    for _ in range(warmup):
+        kla.scan_forward(*args, out=outs, workspace=ws)
+    torch.cuda.synchronize()
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_mod is not None and dist_mod.is_initialized():
+        dist_mod.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        kla.scan_forward(*args, out=outs, workspace=ws)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist_mod is not None and dist_mod.is_initialized():
+        dist_mod.barrier()
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error in the timed region")
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch = [a.elapsed_time(b) for a, b in ev]
+    return total_ms, per_launch
+
+
+def time_e2e(kla, w, host, steps: int):
+    """Public API with pinned HOST tensors: H2D copies, scan, D2H copies, sync."""
+    import torch
+    B, T, H, N = w.B, w.T, w.H, w.N
+    outs = [torch.empty((B, T, H, N), dtype=torch.float32, pin_memory=True) for _ in range(4)]
+    args = (host["a"], host["p"], host["phi"], host["b"], host["lam0"], host["eta0"])
+    kla.scan_forward(*args, out=outs)  # warm-up (allocator, first-touch of pinned pages)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        kla.scan_forward(*args, out=outs)
+    torch.cuda.synchronize()
+    dt = (time.perf_counter() - t0) / steps
+    h2d = sum(host[k].numel() * host[k].element_size() for k in host)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    return dt, h2d, d2h
+
+
+def time_decode(kla, device, steps_tokens: int | None, replays: int):
+    """Decode workload: tokens replayed from a CUDA graph of kla_scan_step calls."""
+    import torch
+    w = wl.WORKLOADS["decode"]
+    if steps_tokens is not None:
+        w = w.with_shape(T=steps_tokens)
+    dev, _ = inputs_to_device(w, device, keep_host=False)
+    steps = {k: dev.pop(k).transpose(0, 1).contiguous() for k in wl.INPUT_NAMES}  # [T, B, H, N]
+    lam = dev["lam0"].clone()
+    eta = dev["eta0"].clone()
+    mu = torch.empty_like(lam)
+    var = torch.empty_like(lam)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for t in range(3):  # warm-up, eager
+            kla.scan_step(steps["a"][t], steps["p"][t], steps["phi"][t], steps["b"][t], lam, eta,
+                          mu_out=mu, var_out=var, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for t in range(w.T):
+            kla.scan_step(steps["a"][t], steps["p"][t], steps["phi"][t], steps["b"][t], lam, eta,
+                          mu_out=mu, var_out=var, stream=s)
+    g.replay()  # warm-up replay
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (replays * w.T)
+    del g
+    tc = w.channels
+    bytes_step = decode_bytes_per_channel(w) * tc
+    return {"workload": w.summary, "ms_per_token": ms, "value": tc / (ms * 1e-3), "unit": UNIT,
+            "gb_per_s": bytes_step / (ms * 1e-3) / 1e9, "bytes_per_token": bytes_step,
+            "tokens_per_replay": w.T, "replays": replays,
+            "note": "one kla_scan_step launch per token; the 8 MB fp32 state can stay L2-resident"}
+
+
+def cpu_oracle_sample(w: wl.Workload, host_arrays, target_s: float = 10.0):
+    """Time the fp64 oracle on a bounded sample of whole channels of the workload."""
+    import oracle
+    threads = os.cpu_count() or 1
+    orc = oracle.default()
+    threads = min(threads, orc.max_threads())
+    HN = w.H * w.N
+
+    def run(nch):
+        idx = np.arange(nch)
+        b_idx, c_idx = np.divmod(idx, HN)
+        x = {k: np.ascontiguousarray(host_arrays[k].reshape(w.B, w.T, HN)[b_idx, :, c_idx].T)
+             .reshape(1, w.T, 1, nch) for k in wl.INPUT_NAMES}
+        t0 = time.perf_counter()
+        orc.forward(x["a"], x["p"], x["phi"], x["b"], np.ones((1, 1, nch)), np.zeros((1, 1, nch)),
+                    threads=threads)
+        return time.perf_counter() - t0
+
+    n = min(w.channels, max(threads, 8))
+    dt = run(n)
+    while dt < target_s / 4 and n < w.channels:
+        n = min(w.channels, int(n * max(2.0, target_s / max(dt, 1e-3) / 2)))
+        dt = run(n)
+    return {"value": n * w.T / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {w.channels} channels x all {w.T} tokens ({n * w.T:,} token-channels), "
+                      f"fp64 sequential covariance-form filter, OpenMP over channels, {dt:.2f} s"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import kalman_linear_attention_b200 as kla
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    base = wl.WORKLOADS[args.workload]
+    w = rank_workload(base, rank)
+    keep_host = not args.no_e2e
+    dev, host = inputs_to_device(w, device, keep_host=keep_host)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    total_ms, per_launch = time_forward(kla, w, dev, args.steps, args.warmup, dist if world > 1 else None)
+    clocks = sampler.stop()
+
+    max_ms = max_over_ranks(total_ms, dist if world > 1 else None)
+    tc_rank = w.token_channels
+    tc_all = tc_rank * world
+    value = tc_all * args.steps / (max_ms * 1e-3)
+    bpt = algorithmic_bytes_per_tc(w)
+    launch_ms = statistics.mean(per_launch)
+    achieved = bpt * tc_rank / (launch_ms * 1e-3) / 1e9
+    peak, peak_src = measured_peaks()
+    traffic = recorded_traffic(args.workload)
+
+    e2e = None
+    if host is not None:
+        del dev
+        torch.cuda.empty_cache()
+        e2e_s, h2d, d2h = time_e2e(kla, w, host, args.e2e_steps)
+        e2e_s = max_over_ranks(e2e_s, dist if world > 1 else None)
+        e2e = {"value": tc_all / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_s * 1e3,
+               "how": "scan_forward on pinned host tensors: H2D of a, p, phi, b, lam0, eta0, "
+                      "the scan, D2H of lambda, eta, mu, var, stream sync; wall clock"}
+    decode = None
+    if not args.no_decode:
+        decode = time_decode(kla, device, None, args.decode_replays)
+        decode["gb_per_s_frac_of_peak"] = decode["gb_per_s"] / peak
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and host is not None:
+        arrays = {k: host[k].float().numpy() for k in wl.INPUT_NAMES}
+        cpu = cpu_oracle_sample(w, arrays)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32" if w.dtype == "f32" else "bf16",
+        "data": "synthetic (seeded numpy draws of the workload's distributions; own seed per rank)",
+        "config": {"workload": f"{base.name}: {base.summary}", "B": base.B, "H": base.H, "N": base.N,
+                   "T": base.T, "token_channels_per_gpu": tc_rank, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 ({bpt // 2 * tc_rank / 1e9:.1f} GB of inputs vs 126 MB L2)"},
+        "gb_per_s": bpt * tc_all * args.steps / (max_ms * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
+                     "traffic": traffic, "algorithmic_bytes_per_launch": bpt * tc_rank,
+                     "kernel": "kla_forward_kernel (+ its workspace clear, timed together)",
+                     "launch_ms": launch_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "decode": decode,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+
+
+# ----------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = wl.WORKLOADS[args.workload]
+    threads = min(os.cpu_count() or 1, oracle.default().max_threads())
+    # a bounded sample per step: whole channels, all tokens
+    nch = max(1, min(w.channels, args.ref_channels))
+    HN = w.H * w.N
+    ws = w.with_shape(B=1, H=1, N=nch) if w.B * HN >= nch else w
+    x = wl.generate(ws.with_shape(T=w.T))
+    a = {k: x[k] for k in wl.INPUT_NAMES}
+    orc = oracle.default()
+    for _ in range(args.warmup):
+        orc.forward(a["a"], a["p"], a["phi"], a["b"], x["lam0"], x["eta0"], threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.forward(a["a"], a["p"], a["phi"], a["b"], x["lam0"], x["eta0"], threads=threads)
+    dt = (time.perf_counter() - t0) / args.steps
+    tc = nch * w.T
+    value = tc / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.summary}", "B": w.B, "H": w.H, "N": w.N, "T": w.T},
+        "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": threads,
+                         "sample": f"{nch} of {w.channels} channels x all {w.T} tokens per step "
+                                   f"(same distributions, seed {w.seed}), fp64 sequential filter"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long", choices=sorted(k for k, v in wl.WORKLOADS.items()
+                                                                  if not v.decode))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--decode-replays", type=int, default=5)
+    ap.add_argument("--ref-channels", type=int, default=256)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

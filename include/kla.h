@@ -1,0 +1,191 @@
+/*
+ * kla.h -- C ABI of the B200 (sm_100a) Kalman Linear Attention filter scan.
+ *
+ * The library computes, for every channel (b, h, n) independently, the scalar
+ * information-form Kalman filter of Kalman Linear Attention (KLA):
+ *
+ *   precision   lambda_t = ((1 + p_t phi_t) lambda_{t-1} + a_t^2 phi_t)
+ *                          / (p_t lambda_{t-1} + a_t^2)
+ *               i.e. the Moebius map of M_t = [[1 + p_t phi_t, a_t^2 phi_t],
+ *                                              [p_t,           a_t^2      ]]
+ *               (Pith review of "Kalman Linear Attention: Parallel Bayesian
+ *                Filtering For Efficient Language Modelling and State
+ *                Tracking", section "What carries the argument"; its
+ *                derivation from the information-form predict / update is
+ *                the review's "Circularity Check", Theorem 1)
+ *   gate        f_t = a_t / (a_t^2 + p_t lambda_{t-1})
+ *   info mean   eta_t = f_t eta_{t-1} + b_t
+ *               (the affine information-mean recursion with the
+ *                precision-ratio forget gate, review "Core claim" and
+ *                Theorem 2)
+ *   outputs     lambda_t, eta_t, mu_t = eta_t / lambda_t, var_t = 1 / lambda_t
+ *               (explicit belief-state uncertainty, review "Core claim" and
+ *                the ICML 2026 poster abstract)
+ *
+ * a_t is the state decay, p_t the process-noise variance, phi_t the
+ * token-evidence precision (k_t^2 Lambda^v_t) and b_t the token information
+ * (k_t Lambda^v_t v_t).  (lambda_0, eta_0) is the prior before token 1; output
+ * row t-1 holds the posterior after token t.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Layout: per-token tensors are [B, T, H, N] row-major (N fastest), dense.
+ *   Per-channel tensors (prior, decode state, one decode token) are
+ *   [B, H, N] row-major, dense.  A "channel" is one (b, h, n).
+ * - Memory: every pointer is DEVICE memory owned by the caller (allocate it
+ *   with cudaMalloc, torch, ...).  The library allocates nothing and keeps no
+ *   pointer after a call returns.
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *   default stream).  Calls enqueue work and return without synchronising;
+ *   results are valid once the stream reaches that point.
+ * - Errors: argument errors are detected on the host before anything is
+ *   enqueued and return a kla_status_t != KLA_OK; nothing is written then.
+ *   A launch failure returns KLA_ERR_CUDA.  Device-side failures (a bounded
+ *   wait that ran out) are recorded on the device and reported by
+ *   kla_get_error(); the affected outputs are NaN.
+ * - Preconditions, not checked per element: p_t >= 0, phi_t >= 0,
+ *   lambda_0 > 0, and a_t^2 + p_t lambda_{t-1} > 0 (e.g. a_t != 0 or p_t > 0).
+ *   Any real a_t is allowed (only a_t^2 enters the precision; the sign of a_t
+ *   enters the gate).
+ * - Arithmetic: inputs are fp32 or bf16 (converted exactly to fp32 on load);
+ *   state and outputs are fp32 with IEEE division; no fast-math.
+ * - Outputs must not overlap inputs or each other.
+ */
+#ifndef KLA_H
+#define KLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KLA_ABI_VERSION 1
+
+typedef enum {
+    KLA_F32 = 0,  /* IEEE binary32 */
+    KLA_BF16 = 1  /* bfloat16 (8-bit exponent, 7-bit mantissa) */
+} kla_dtype_t;
+
+typedef enum {
+    KLA_OK = 0,
+    KLA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, overlap, size overflow */
+    KLA_ERR_UNSUPPORTED_DTYPE = 2,   /* dtype is not KLA_F32 / KLA_BF16 */
+    KLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the required size */
+    KLA_ERR_CUDA = 4,                /* a CUDA runtime / driver call failed */
+    KLA_ERR_TIMEOUT = 5,             /* a device-side bounded wait ran out */
+    KLA_ERR_MISALIGNED = 6           /* workspace not 256-byte aligned */
+} kla_status_t;
+
+/* ABI version of the loaded library (KLA_ABI_VERSION it was built with). */
+int kla_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kla_strerror(kla_status_t status);
+
+/*
+ * Size in bytes of the device workspace that kla_scan_forward needs for a
+ * problem of this shape and input dtype, written to *bytes.  The workspace
+ * holds the cross-chunk carries of the scan (per chunk and channel: a 3x3
+ * homogeneous aggregate and the inclusive state) and their ready flags.
+ * Returns KLA_ERR_INVALID_ARG for negative sizes or a null `bytes`.
+ */
+kla_status_t kla_scan_forward_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                             kla_dtype_t in_dtype, size_t *bytes);
+
+/*
+ * Forward filter over whole sequences (the parallel scan; review "Core claim":
+ * both recursions compose associatively, O(T) work).
+ *
+ *   a, p, phi, b   [B, T, H, N] inputs of dtype in_dtype (device, read only)
+ *   lambda0, eta0  [B, H, N] fp32 prior (device, read only)
+ *   lambda_out     [B, T, H, N] fp32 posterior precision (device, written)
+ *   eta_out        [B, T, H, N] fp32 information mean (device, written)
+ *   mu_out         [B, T, H, N] fp32 posterior mean, or NULL to skip
+ *   var_out        [B, T, H, N] fp32 posterior variance, or NULL to skip
+ *   workspace      device scratch of at least
+ *                  kla_scan_forward_workspace_size(...) bytes, 256-byte
+ *                  aligned; its contents on entry do not matter and are
+ *                  undefined on return.  Two calls in flight at the same time
+ *                  (e.g. on two streams) need two workspaces.
+ *
+ * T == 0 or B*H*N == 0 is a valid empty problem (nothing is enqueued).
+ * The last row of lambda_out / eta_out is the state to continue decoding from
+ * with kla_scan_step.
+ */
+kla_status_t kla_scan_forward(const void *a, const void *p, const void *phi, const void *b,
+                              kla_dtype_t in_dtype,
+                              const float *lambda0, const float *eta0,
+                              float *lambda_out, float *eta_out, float *mu_out, float *var_out,
+                              int64_t B, int64_t T, int64_t H, int64_t N,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decode token for every channel (constant work per token;
+ * the running posterior is a sufficient summary: "Kalman filter" primer
+ * section 6.2, and the review's O(1)-per-step recurrent form).
+ *
+ *   a, p, phi, b   [B, H, N] inputs of this token, dtype in_dtype (read only)
+ *   lambda_state   [B, H, N] fp32 precision, read and overwritten in place
+ *   eta_state      [B, H, N] fp32 information mean, read and overwritten
+ *   mu_out         [B, H, N] fp32 posterior mean of this token, or NULL
+ *   var_out        [B, H, N] fp32 posterior variance of this token, or NULL
+ *
+ * B*H*N == 0 is valid (nothing is enqueued).  The state pointers may not
+ * overlap the inputs or the other outputs.
+ */
+kla_status_t kla_scan_step(const void *a, const void *p, const void *phi, const void *b,
+                           kla_dtype_t in_dtype,
+                           float *lambda_state, float *eta_state,
+                           float *mu_out, float *var_out,
+                           int64_t B, int64_t H, int64_t N, void *stream);
+
+/*
+ * Synchronise `stream`, then report the first failure since the previous
+ * call on the current device: KLA_ERR_CUDA for a CUDA error (sticky or not),
+ * KLA_ERR_TIMEOUT if a kernel's bounded wait ran out (the outputs that
+ * depended on it are NaN), KLA_OK otherwise.  Clears the device-side record.
+ */
+kla_status_t kla_get_error(void *stream);
+
+/*
+ * Upper bound, in nanoseconds, of every device-side wait (a chunk waiting for
+ * the carry of its predecessor; a CTA waiting for its own tile load).  The
+ * default is 1e9 (one second).  A wait that runs out records KLA_ERR_TIMEOUT
+ * and writes NaN instead of blocking.  Applies to calls enqueued afterwards.
+ * Returns KLA_ERR_INVALID_ARG for 0.
+ */
+kla_status_t kla_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Test hook for the failure path: enqueue one kernel on `stream` that waits,
+ * through the same bounded wait the scan uses, on a device flag that nothing
+ * ever sets, with the current wait limit.  The wait runs out, records
+ * KLA_ERR_TIMEOUT, and the kernel returns; kla_get_error() then reports it.
+ */
+kla_status_t kla_debug_unset_flag_wait(void *stream);
+
+/*
+ * Number of tokens in one chunk of the forward scan (the unit of the
+ * cross-chunk carry).  Informational; results do not depend on it.
+ */
+int kla_forward_chunk_tokens(void);
+
+/*
+ * Test hook for the forward scan's failure path: in kla_scan_forward calls
+ * enqueued afterwards, the chunks with index `chunk` (tokens
+ * [chunk * kla_forward_chunk_tokens(), ...)) wait for their carry on a device
+ * flag that nothing sets, instead of on the preceding chunk.  The wait runs
+ * out after the wait limit, records KLA_ERR_TIMEOUT and writes NaN for that
+ * chunk.  Earlier chunks are unaffected; a later chunk is either exact (its
+ * look-back composed the stalled chunk's published aggregate) or NaN (it read
+ * the stalled chunk's poisoned carry).  -1 (the default) turns the hook off.
+ */
+kla_status_t kla_debug_stall_chunk(int64_t chunk);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KLA_H */

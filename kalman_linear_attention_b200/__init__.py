@@ -1,1 +1,20 @@
-"""B200-native Kalman Linear Attention filter scan (binding added with the CUDA library)."""
+"""B200-native (sm_100a) information-form Kalman filter scan of Kalman Linear
+Attention (KLA).
+
+The compute path is the C-ABI CUDA library ``libkla.so`` (declared in
+``include/kla.h``); :mod:`.api` is its thin ctypes binding and is imported on
+first use, so that importing :mod:`.workloads` (seeded inputs) needs neither
+torch nor the built library.
+"""
+_API_NAMES = {
+    "scan_forward", "scan_step", "workspace_size", "new_workspace", "get_error",
+    "set_wait_limit_ns", "debug_unset_flag_wait", "debug_stall_chunk", "chunk_tokens",
+    "KlaError", "lib", "load_library",
+}
+
+
+def __getattr__(name):
+    if name in _API_NAMES:
+        from . import api
+        return getattr(api, name)
+    raise AttributeError(name)

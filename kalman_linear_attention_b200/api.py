@@ -1,0 +1,233 @@
+"""Thin Python binding of the C ABI in ``include/kla.h`` (ctypes).
+
+Argument marshalling only: every step of the filter runs in the CUDA kernels
+of ``libkla.so``.  PyTorch is used for device memory and streams.  There is no
+CPU fallback: without the built library, or without a CUDA device, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libkla.so")
+
+KLA_F32 = 0
+KLA_BF16 = 1
+STATUS = {0: "KLA_OK", 1: "KLA_ERR_INVALID_ARG", 2: "KLA_ERR_UNSUPPORTED_DTYPE",
+          3: "KLA_ERR_WORKSPACE_TOO_SMALL", 4: "KLA_ERR_CUDA", 5: "KLA_ERR_TIMEOUT",
+          6: "KLA_ERR_MISALIGNED"}
+KLA_OK, KLA_ERR_INVALID_ARG, KLA_ERR_UNSUPPORTED_DTYPE = 0, 1, 2
+KLA_ERR_WORKSPACE_TOO_SMALL, KLA_ERR_CUDA, KLA_ERR_TIMEOUT, KLA_ERR_MISALIGNED = 3, 4, 5, 6
+
+# Every exported symbol of include/kla.h, with (restype, argtypes).
+_VP, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+SIGNATURES = {
+    "kla_abi_version": (ctypes.c_int, []),
+    "kla_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "kla_scan_forward_workspace_size": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int,
+                                                       ctypes.POINTER(_SZ)]),
+    "kla_scan_forward": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP,
+                                        _VP, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
+    "kla_scan_step": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
+                                     _I64, _I64, _I64, _VP]),
+    "kla_get_error": (ctypes.c_int, [_VP]),
+    "kla_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
+    "kla_debug_unset_flag_wait": (ctypes.c_int, [_VP]),
+    "kla_forward_chunk_tokens": (ctypes.c_int, []),
+    "kla_debug_stall_chunk": (ctypes.c_int, [_I64]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class KlaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+def load_library(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load ``libkla.so`` and declare the C signatures (raises if it is missing)."""
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is not built; build it with "
+            "`python -m kalman_linear_attention_b200._build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != KLA_OK:
+        raise KlaError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KLA_F32
+    if t.dtype == torch.bfloat16:
+        return KLA_BF16
+    raise TypeError(f"inputs must be float32 or bfloat16, got {t.dtype}")
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _require_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensor must be on a CUDA device")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensor must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def workspace_size(B: int, T: int, H: int, N: int, dtype: torch.dtype = torch.float32) -> int:
+    code = KLA_BF16 if dtype == torch.bfloat16 else KLA_F32
+    out = ctypes.c_size_t(0)
+    _check(lib().kla_scan_forward_workspace_size(B, T, H, N, code, ctypes.byref(out)),
+           "kla_scan_forward_workspace_size")
+    return int(out.value)
+
+
+def chunk_tokens() -> int:
+    return int(lib().kla_forward_chunk_tokens())
+
+
+def new_workspace(B: int, T: int, H: int, N: int, dtype: torch.dtype, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(workspace_size(B, T, H, N, dtype), 1), dtype=torch.uint8, device=device)
+
+
+def scan_forward(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.Tensor,
+                 lam0: torch.Tensor, eta0: torch.Tensor, *,
+                 want_mu: bool = True, want_var: bool = True,
+                 out: Optional[Sequence[Optional[torch.Tensor]]] = None,
+                 workspace: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None,
+                 ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
+    """Filter [B, T, H, N] inputs from the [B, H, N] prior.
+
+    Returns (lambda, eta, mu, var) as fp32 [B, T, H, N] tensors (mu / var are
+    None when not wanted).  CUDA inputs give CUDA outputs, enqueued on
+    ``stream`` (default: the current stream) without synchronising.  CPU
+    inputs (ideally pinned) are copied to the current CUDA device, filtered
+    there, and copied back; the call then returns CPU tensors after a
+    synchronise.  ``out`` may supply the four output tensors (None entries
+    for skipped outputs) on the side the results are returned on.
+    """
+    if not (a.shape == p.shape == phi.shape == b.shape) or a.dim() != 4:
+        raise ValueError("a, p, phi, b must share one [B, T, H, N] shape")
+    if not (a.dtype == p.dtype == phi.dtype == b.dtype):
+        raise TypeError("a, p, phi, b must share one dtype")
+    B, T, H, N = a.shape
+    if lam0.shape != (B, H, N) or eta0.shape != (B, H, N):
+        raise ValueError("lam0 and eta0 must be [B, H, N]")
+    if lam0.dtype != torch.float32 or eta0.dtype != torch.float32:
+        raise TypeError("lam0 and eta0 must be float32")
+    host = not a.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        nb = a.is_pinned()
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(s):
+            d_in = [x.to(dev, non_blocking=nb) for x in (a, p, phi, b, lam0, eta0)]
+            d_out = scan_forward(*d_in, want_mu=want_mu, want_var=want_var, stream=s,
+                                 workspace=workspace)
+            res = []
+            for i, d in enumerate(d_out):
+                if d is None:
+                    res.append(None)
+                    continue
+                dst = out[i] if out is not None and out[i] is not None else \
+                    torch.empty(d.shape, dtype=d.dtype, pin_memory=nb)
+                dst.copy_(d, non_blocking=nb)
+                res.append(dst)
+        s.synchronize()
+        return tuple(res)
+
+    _require_cuda(a, p, phi, b, lam0, eta0)
+    code = _dtype_code(a)
+    dev = a.device
+    if out is None:
+        outs = [torch.empty((B, T, H, N), dtype=torch.float32, device=dev),
+                torch.empty((B, T, H, N), dtype=torch.float32, device=dev),
+                torch.empty((B, T, H, N), dtype=torch.float32, device=dev) if want_mu else None,
+                torch.empty((B, T, H, N), dtype=torch.float32, device=dev) if want_var else None]
+    else:
+        outs = list(out)
+        _require_cuda(*[o for o in outs if o is not None])
+    if workspace is None:
+        workspace = new_workspace(B, T, H, N, a.dtype, dev)
+    with torch.cuda.device(dev):
+        st = kla_scan_forward_raw(a, p, phi, b, code, lam0, eta0, outs, B, T, H, N, workspace,
+                                  _stream_handle(stream))
+    _check(st, "kla_scan_forward")
+    return tuple(outs)
+
+
+def kla_scan_forward_raw(a, p, phi, b, code, lam0, eta0, outs, B, T, H, N, workspace, stream) -> int:
+    """Direct C-ABI call; returns the status code."""
+    return lib().kla_scan_forward(
+        _ptr(a), _ptr(p), _ptr(phi), _ptr(b), code, _ptr(lam0), _ptr(eta0),
+        _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), B, T, H, N,
+        _ptr(workspace), workspace.numel() if workspace is not None else 0, stream)
+
+
+def scan_step(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.Tensor,
+              lam_state: torch.Tensor, eta_state: torch.Tensor, *,
+              mu_out: Optional[torch.Tensor] = None, var_out: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> None:
+    """One decode token for every channel of [B, H, N] inputs; updates
+    ``lam_state`` / ``eta_state`` in place and writes ``mu_out`` / ``var_out``
+    when given.  Enqueued on ``stream`` (default: the current stream)."""
+    if not (a.shape == p.shape == phi.shape == b.shape == lam_state.shape == eta_state.shape):
+        raise ValueError("step inputs and state must share one [B, H, N] shape")
+    if a.dim() != 3:
+        raise ValueError("step tensors are [B, H, N]")
+    if lam_state.dtype != torch.float32 or eta_state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    _require_cuda(a, p, phi, b, lam_state, eta_state, mu_out, var_out)
+    B, H, N = a.shape
+    with torch.cuda.device(a.device):
+        st = lib().kla_scan_step(_ptr(a), _ptr(p), _ptr(phi), _ptr(b), _dtype_code(a),
+                                 _ptr(lam_state), _ptr(eta_state), _ptr(mu_out), _ptr(var_out),
+                                 B, H, N, _stream_handle(stream))
+    _check(st, "kla_scan_step")
+
+
+def get_error(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise and return the device-side status (KLA_OK, KLA_ERR_TIMEOUT, ...)."""
+    return int(lib().kla_get_error(_stream_handle(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _check(lib().kla_set_wait_limit_ns(int(ns)), "kla_set_wait_limit_ns")
+
+
+def debug_unset_flag_wait(stream: Optional[torch.cuda.Stream] = None) -> None:
+    _check(lib().kla_debug_unset_flag_wait(_stream_handle(stream)), "kla_debug_unset_flag_wait")
+
+
+def debug_stall_chunk(chunk: int) -> None:
+    _check(lib().kla_debug_stall_chunk(int(chunk)), "kla_debug_stall_chunk")

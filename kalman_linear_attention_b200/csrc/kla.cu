@@ -1,0 +1,359 @@
+// kla.cu -- host side of the C ABI declared in include/kla.h: argument
+// checks, workspace layout, TMA tensor maps and kernel launches.  Every step
+// of the filter runs in the kernels of kla_forward.cuh / kla_step.cuh; this
+// file only validates, describes memory and launches.
+#include "kla.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "kla_forward.cuh"
+#include "kla_step.cuh"
+
+#define KLA_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+using kla::FwdMaps;
+using kla::FwdParams;
+using kla::StepParams;
+
+// Tile geometry of the forward scan: L tokens x CW channels per CTA, R rows
+// of threads (S = L / R tokens per thread).
+constexpr int kL = 64;
+constexpr int kCW = 64;
+constexpr int kR = 4;
+constexpr int kNW = kCW / 32;
+
+constexpr size_t kHeaderBytes = 256;  // ticket counter + padding
+constexpr int kMaxGrid = 0x7fffffff;
+
+std::atomic<uint64_t> g_wait_ns{1000000000ull};
+std::atomic<int64_t> g_stall_chunk{-1};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+size_t dtype_size(kla_dtype_t d) { return d == KLA_BF16 ? 2 : 4; }
+
+bool dtype_ok(kla_dtype_t d) { return d == KLA_F32 || d == KLA_BF16; }
+
+struct Range {
+    uintptr_t lo, hi;
+};
+
+bool overlaps(const Range &x, const Range &y) {
+    return x.lo < y.hi && y.lo < x.hi;
+}
+
+// Any two of `outs` overlap, or any output overlaps any input.
+bool any_overlap(const Range *outs, int n_out, const Range *ins, int n_in) {
+    for (int i = 0; i < n_out; ++i) {
+        if (outs[i].lo == outs[i].hi) continue;
+        for (int j = i + 1; j < n_out; ++j)
+            if (outs[j].lo != outs[j].hi && overlaps(outs[i], outs[j])) return true;
+        for (int j = 0; j < n_in; ++j)
+            if (ins[j].lo != ins[j].hi && overlaps(outs[i], ins[j])) return true;
+    }
+    return false;
+}
+
+Range range_of(const void *p, int64_t bytes) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    return Range{lo, p ? lo + (uintptr_t)bytes : lo};
+}
+
+// Workspace layout of one forward call.
+struct FwdLayout {
+    int64_t nct = 0, nchunks = 0, tiles = 0;
+    size_t flags_off = 0, agg_off = 0, incl_off = 0, clear_bytes = 0, total = 0;
+};
+
+bool fwd_layout(int64_t B, int64_t T, int64_t HN, FwdLayout *lay) {
+    lay->nct = (HN + kCW - 1) / kCW;
+    lay->nchunks = (T + kL - 1) / kL;
+    int64_t bt = 0, tiles = 0;
+    if (!mul_ok(B, lay->nct, &bt) || !mul_ok(bt, lay->nchunks, &tiles)) return false;
+    if (tiles > kMaxGrid) return false;
+    lay->tiles = tiles;
+    lay->flags_off = kHeaderBytes;
+    const size_t flags_bytes = round_up((size_t)tiles * kNW * sizeof(unsigned), 256);
+    lay->agg_off = lay->flags_off + flags_bytes;
+    lay->incl_off = lay->agg_off + round_up((size_t)tiles * 7 * kCW * sizeof(float), 256);
+    lay->total = lay->incl_off + round_up((size_t)tiles * 2 * kCW * sizeof(float), 256);
+    lay->clear_bytes = kHeaderBytes + flags_bytes;
+    return true;
+}
+
+// ---- TMA tensor maps --------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// [B, T, HN] tensor viewed as dims {HN, T, B}, box {kCW, kL, 1}.
+bool encode_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz,
+                int64_t B, int64_t T, int64_t HN) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)HN, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)(HN * esz), (cuuint64_t)(T * HN * esz)};
+    const cuuint32_t box[3] = {(cuuint32_t)kCW, (cuuint32_t)kL, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- per-device launch attributes ------------------------------------------
+template <typename K>
+cudaError_t ensure_smem_attr(K kernel, int smem) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void *>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kernel));
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count(key)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) done.insert(key);
+    return e;
+}
+
+template <typename Tin, bool TMA>
+cudaError_t launch_forward(const FwdParams &prm, const FwdMaps &maps, int64_t tiles,
+                           cudaStream_t stream) {
+    using Cfg = kla::FwdTile<Tin, kL, kCW, kR>;
+    auto kernel = kla::kla_forward_kernel<Tin, kL, kCW, kR, TMA>;
+    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    kernel<<<(unsigned)tiles, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_clear(void *ws, size_t bytes, cudaStream_t stream) {
+    const int64_t n16 = (int64_t)(bytes / 16);
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>((n16 + threads - 1) / threads, 148 * 8);
+    kla::kla_clear_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), threads, 0, stream>>>(
+        static_cast<uint4 *>(ws), n16);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+KLA_API int kla_abi_version(void) { return KLA_ABI_VERSION; }
+
+KLA_API const char *kla_strerror(kla_status_t s) {
+    switch (s) {
+        case KLA_OK: return "KLA_OK";
+        case KLA_ERR_INVALID_ARG: return "KLA_ERR_INVALID_ARG: invalid argument";
+        case KLA_ERR_UNSUPPORTED_DTYPE: return "KLA_ERR_UNSUPPORTED_DTYPE: dtype must be KLA_F32 or KLA_BF16";
+        case KLA_ERR_WORKSPACE_TOO_SMALL: return "KLA_ERR_WORKSPACE_TOO_SMALL: workspace below the required size";
+        case KLA_ERR_CUDA: return "KLA_ERR_CUDA: a CUDA call failed";
+        case KLA_ERR_TIMEOUT: return "KLA_ERR_TIMEOUT: a device-side bounded wait ran out";
+        case KLA_ERR_MISALIGNED: return "KLA_ERR_MISALIGNED: workspace must be 256-byte aligned";
+    }
+    return "unknown kla_status_t";
+}
+
+KLA_API kla_status_t kla_scan_forward_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                                     kla_dtype_t in_dtype, size_t *bytes) {
+    if (!bytes || B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0;
+    if (!mul_ok(H, N, &HN)) return KLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || HN == 0) {
+        *bytes = 0;
+        return KLA_OK;
+    }
+    FwdLayout lay;
+    if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
+    *bytes = lay.total;
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *phi, const void *b,
+                                      kla_dtype_t in_dtype, const float *lambda0, const float *eta0,
+                                      float *lambda_out, float *eta_out, float *mu_out,
+                                      float *var_out, int64_t B, int64_t T, int64_t H, int64_t N,
+                                      void *workspace, size_t workspace_bytes, void *stream) {
+    if (B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, C = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, HN, &C) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems))
+        return KLA_ERR_INVALID_ARG;
+    if (elems == 0) return KLA_OK;
+    if (!a || !p || !phi || !b || !lambda0 || !eta0 || !lambda_out || !eta_out)
+        return KLA_ERR_INVALID_ARG;
+    const size_t esz = dtype_size(in_dtype);
+    int64_t in_bytes = 0, out_bytes = 0;
+    if (!mul_ok(elems, (int64_t)esz, &in_bytes) || !mul_ok(elems, 4, &out_bytes))
+        return KLA_ERR_INVALID_ARG;
+    const Range outs[4] = {range_of(lambda_out, out_bytes), range_of(eta_out, out_bytes),
+                           range_of(mu_out, out_bytes), range_of(var_out, out_bytes)};
+    const Range ins[7] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(phi, in_bytes),
+                          range_of(b, in_bytes), range_of(lambda0, C * 4), range_of(eta0, C * 4),
+                          range_of(workspace, (int64_t)workspace_bytes)};
+    if (any_overlap(outs, 4, ins, 7)) return KLA_ERR_INVALID_ARG;
+
+    FwdLayout lay;
+    if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < lay.total) return KLA_ERR_WORKSPACE_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KLA_ERR_MISALIGNED;
+    if (T > INT32_MAX || HN > INT32_MAX || B > INT32_MAX || lay.nct > INT32_MAX ||
+        lay.nchunks > INT32_MAX)
+        return KLA_ERR_INVALID_ARG;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    FwdParams prm;
+    prm.in[0] = a; prm.in[1] = p; prm.in[2] = phi; prm.in[3] = b;
+    prm.lam0 = lambda0; prm.eta0 = eta0;
+    prm.out[0] = lambda_out; prm.out[1] = eta_out; prm.out[2] = mu_out; prm.out[3] = var_out;
+    prm.T = T; prm.HN = HN;
+    prm.tiles_per_chunk = B * lay.nct;
+    prm.nct = (int)lay.nct;
+    prm.nchunks = (int)lay.nchunks;
+    prm.ticket = reinterpret_cast<unsigned *>(ws);
+    prm.flags = reinterpret_cast<unsigned *>(ws + lay.flags_off);
+    prm.agg_ws = reinterpret_cast<float *>(ws + lay.agg_off);
+    prm.incl_ws = reinterpret_cast<float *>(ws + lay.incl_off);
+    prm.wait_ns = g_wait_ns.load();
+    prm.stall_chunk = g_stall_chunk.load();
+
+    // TMA boxes when the geometry allows them; plain loads otherwise.
+    FwdMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    bool tma = (HN * (int64_t)esz) % 16 == 0 && T >= kL && HN >= kCW;
+    const void *ptrs[8] = {a, p, phi, b, lambda_out, eta_out, mu_out, var_out};
+    for (int k = 0; k < 8 && tma; ++k)
+        if (ptrs[k] && !aligned16(ptrs[k])) tma = false;
+    if (tma) {
+        const CUtensorMapDataType dt =
+            in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        for (int k = 0; k < 4 && tma; ++k) tma = encode_map(&maps.in[k], ptrs[k], dt, esz, B, T, HN);
+        for (int k = 0; k < 4 && tma; ++k)
+            if (ptrs[4 + k])
+                tma = encode_map(&maps.out[k], ptrs[4 + k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN);
+    }
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_clear(ws, lay.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
+    cudaError_t e;
+    if (in_dtype == KLA_F32)
+        e = tma ? launch_forward<float, true>(prm, maps, lay.tiles, st)
+                : launch_forward<float, false>(prm, maps, lay.tiles, st);
+    else
+        e = tma ? launch_forward<__nv_bfloat16, true>(prm, maps, lay.tiles, st)
+                : launch_forward<__nv_bfloat16, false>(prm, maps, lay.tiles, st);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+KLA_API kla_status_t kla_scan_step(const void *a, const void *p, const void *phi, const void *b,
+                                   kla_dtype_t in_dtype, float *lambda_state, float *eta_state,
+                                   float *mu_out, float *var_out, int64_t B, int64_t H, int64_t N,
+                                   void *stream) {
+    if (B < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, C = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, HN, &C)) return KLA_ERR_INVALID_ARG;
+    if (C == 0) return KLA_OK;
+    if (!a || !p || !phi || !b || !lambda_state || !eta_state) return KLA_ERR_INVALID_ARG;
+    const size_t esz = dtype_size(in_dtype);
+    int64_t in_bytes = 0, st_bytes = 0;
+    if (!mul_ok(C, (int64_t)esz, &in_bytes) || !mul_ok(C, 4, &st_bytes)) return KLA_ERR_INVALID_ARG;
+    const Range outs[4] = {range_of(lambda_state, st_bytes), range_of(eta_state, st_bytes),
+                           range_of(mu_out, st_bytes), range_of(var_out, st_bytes)};
+    const Range ins[4] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(phi, in_bytes),
+                          range_of(b, in_bytes)};
+    if (any_overlap(outs, 4, ins, 4)) return KLA_ERR_INVALID_ARG;
+
+    StepParams prm;
+    prm.in[0] = a; prm.in[1] = p; prm.in[2] = phi; prm.in[3] = b;
+    prm.lam = lambda_state; prm.eta = eta_state; prm.mu = mu_out; prm.var = var_out;
+    prm.C = C;
+
+    const uintptr_t in_align = esz == 4 ? 15u : 7u;
+    bool vec = (C % 4) == 0;
+    const void *ins_p[4] = {a, p, phi, b};
+    for (int k = 0; k < 4; ++k)
+        if (reinterpret_cast<uintptr_t>(ins_p[k]) & in_align) vec = false;
+    const void *outs_p[4] = {lambda_state, eta_state, mu_out, var_out};
+    for (int k = 0; k < 4; ++k)
+        if (outs_p[k] && !aligned16(outs_p[k])) vec = false;
+
+    const int threads = 256;
+    const int64_t work = vec ? C / 4 : C;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((work + threads - 1) / threads, 148 * 16));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (in_dtype == KLA_F32) {
+        if (vec) kla::kla_step_vec4_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(prm);
+        else kla::kla_step_scalar_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(prm);
+    } else {
+        if (vec) kla::kla_step_vec4_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(prm);
+        else kla::kla_step_scalar_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(prm);
+    }
+    return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+KLA_API kla_status_t kla_get_error(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KLA_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return KLA_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpyFromSymbol(&word, kla::g_error_word, sizeof(word)) != cudaSuccess) return KLA_ERR_CUDA;
+    if (word == 0u) return KLA_OK;
+    const unsigned zero = 0u;
+    if (cudaMemcpyToSymbol(kla::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return KLA_ERR_CUDA;
+    return KLA_ERR_TIMEOUT;
+}
+
+KLA_API kla_status_t kla_set_wait_limit_ns(uint64_t ns) {
+    if (ns == 0) return KLA_ERR_INVALID_ARG;
+    g_wait_ns.store(ns);
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_debug_unset_flag_wait(void *stream) {
+    kla::kla_unset_flag_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_ns.load());
+    return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+KLA_API int kla_forward_chunk_tokens(void) { return kL; }
+
+KLA_API kla_status_t kla_debug_stall_chunk(int64_t chunk) {
+    if (chunk < -1) return KLA_ERR_INVALID_ARG;
+    g_stall_chunk.store(chunk);
+    return KLA_OK;
+}

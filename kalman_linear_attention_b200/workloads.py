@@ -28,6 +28,7 @@ sigmoid(x) = 1/(1+e^-x); all evaluated in fp64):
 from __future__ import annotations
 
 import dataclasses
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 from typing import Dict, Iterator, Tuple
 
@@ -145,17 +146,21 @@ def iter_rows(w: Workload, rows_per_block: int | None = None
     if rows_per_block is None:
         rows_per_block = max(1, _BLOCK_ELEMS // max(HN, 1))
     rngs = _streams(w.seed)
-    r0 = 0
-    while r0 < rows:
-        r1 = min(rows, r0 + rows_per_block)
-        out = {}
-        for name, rng in zip(INPUT_NAMES, rngs):
-            x = _draw(w.dist, name, rng, (r1 - r0) * HN).astype(np.float32)
-            if w.dtype == "bf16":
-                x = round_to_bf16(x)
-            out[name] = x.reshape(r1 - r0, w.H, w.N)
-        yield r0, r1, out
-        r0 = r1
+
+    def one(name, rng, n):
+        x = _draw(w.dist, name, rng, n).astype(np.float32)
+        return round_to_bf16(x) if w.dtype == "bf16" else x
+
+    # the four streams are independent: draw them in parallel (numpy releases the GIL)
+    with ThreadPoolExecutor(max_workers=len(INPUT_NAMES)) as pool:
+        r0 = 0
+        while r0 < rows:
+            r1 = min(rows, r0 + rows_per_block)
+            n = (r1 - r0) * HN
+            futs = [pool.submit(one, name, rng, n) for name, rng in zip(INPUT_NAMES, rngs)]
+            out = {name: f.result().reshape(r1 - r0, w.H, w.N) for name, f in zip(INPUT_NAMES, futs)}
+            yield r0, r1, out
+            r0 = r1
 
 
 def generate(w: Workload) -> Dict[str, np.ndarray]:

@@ -1,0 +1,94 @@
+"""The C-ABI library loads and exports every symbol of include/kla.h; host-side
+argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kla_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kalman_linear_attention_b200 import _build, api
+    _build.build()
+    return api.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from kalman_linear_attention_b200 import api
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(api.SIGNATURES), "binding and header disagree"
+
+
+def test_abi_version(lib):
+    src = open(os.path.join(ROOT, "include", "kla.h")).read()
+    v = int(re.search(r"#define KLA_ABI_VERSION (\d+)", src).group(1))
+    assert lib.kla_abi_version() == v
+
+
+def test_strerror(lib):
+    for code in range(7):
+        assert lib.kla_strerror(code)
+    assert b"unknown" in lib.kla_strerror(99)
+
+
+def test_workspace_size(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.kla_scan_forward_workspace_size(1, 65536, 32, 128, 0, ctypes.byref(out)) == 0
+    L = lib.kla_forward_chunk_tokens()
+    chunks = 65536 // L
+    tiles = chunks * (4096 // 64)
+    # carries: 7 + 2 floats per channel per chunk, plus flags and a header
+    assert out.value >= tiles * 64 * 9 * 4
+    assert out.value < 0.05 * (65536 * 4096 * 32)
+    assert lib.kla_scan_forward_workspace_size(-1, 1, 1, 1, 0, ctypes.byref(out)) == 1
+    assert lib.kla_scan_forward_workspace_size(1, 1, 1, 1, 7, ctypes.byref(out)) == 2
+    assert lib.kla_scan_forward_workspace_size(1, 1, 1, 1, 0, None) == 1
+    assert lib.kla_scan_forward_workspace_size(0, 100, 1, 1, 0, ctypes.byref(out)) == 0
+    assert out.value == 0
+
+
+def test_host_argument_errors(lib):
+    """Rejected before any CUDA call: negative sizes, bad dtype, null pointers,
+    overlapping outputs, small or misaligned workspace; empty problems are OK."""
+    fwd = lib.kla_scan_forward
+    P = 1 << 20  # fake, never dereferenced: every case returns before a launch
+    args = lambda **kw: [kw.get("a", P), kw.get("p", 2 * P), kw.get("phi", 3 * P), kw.get("b", 4 * P),
+                         kw.get("dt", 0), kw.get("lam0", 5 * P), kw.get("eta0", 6 * P),
+                         kw.get("lam", 7 * P), kw.get("eta", 8 * P), kw.get("mu", None),
+                         kw.get("var", None), kw.get("B", 1), kw.get("T", 4), kw.get("H", 1),
+                         kw.get("N", 4), kw.get("ws", 16 * P), kw.get("wsb", 1 << 20), None]
+    assert fwd(*args(B=-1)) == 1
+    assert fwd(*args(dt=3)) == 2
+    assert fwd(*args(a=None)) == 1
+    assert fwd(*args(lam=None)) == 1
+    assert fwd(*args(eta=7 * P)) == 1          # eta_out overlaps lambda_out
+    assert fwd(*args(mu=P)) == 1               # mu_out overlaps input a
+    assert fwd(*args(wsb=16)) == 3             # workspace too small
+    assert fwd(*args(ws=None)) == 3
+    assert fwd(*args(ws=16 * P + 8)) == 6      # misaligned workspace
+    assert fwd(*args(T=0)) == 0                # empty: nothing enqueued
+    assert fwd(*args(B=0, a=None)) == 0
+    step = lib.kla_scan_step
+    sargs = lambda **kw: [kw.get("a", P), kw.get("p", 2 * P), kw.get("phi", 3 * P), kw.get("b", 4 * P),
+                          kw.get("dt", 0), kw.get("lam", 5 * P), kw.get("eta", 6 * P),
+                          kw.get("mu", None), kw.get("var", None), kw.get("B", 1), kw.get("H", 1),
+                          kw.get("N", 4), None]
+    assert step(*sargs(N=-2)) == 1
+    assert step(*sargs(dt=9)) == 2
+    assert step(*sargs(lam=None)) == 1
+    assert step(*sargs(eta=5 * P)) == 1
+    assert step(*sargs(B=0)) == 0
+    assert lib.kla_set_wait_limit_ns(0) == 1
+    assert lib.kla_debug_stall_chunk(-5) == 1

@@ -1,0 +1,61 @@
+"""Failure path on the GPU: bounded waits run out, report KLA_ERR_TIMEOUT, and
+leave the context usable.  Nothing here faults, traps or hangs the GPU: the
+waits target a device word that nothing sets and give up after a short limit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from kalman_linear_attention_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture
+def kla():
+    import kalman_linear_attention_b200 as kla
+    kla.set_wait_limit_ns(2_000_000)  # 2 ms
+    yield kla
+    kla.debug_stall_chunk(-1)
+    kla.set_wait_limit_ns(1_000_000_000)
+
+
+def test_unset_flag_wait_reports_timeout(kla):
+    assert kla.get_error() == 0
+    kla.debug_unset_flag_wait()
+    assert kla.get_error() == 5  # KLA_ERR_TIMEOUT
+    assert kla.get_error() == 0  # cleared
+
+
+def test_stalled_chunk_poisons_only_what_depends_on_it(kla):
+    L = kla.chunk_tokens()
+    w = wl.WORKLOADS["tiny"]  # T = 256 = 4 chunks of 64
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
+    stall = 2
+    kla.debug_stall_chunk(stall)
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    assert kla.get_error() == 5
+    kla.debug_stall_chunk(-1)
+    lam = out[0].double().cpu().numpy()
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    cut = stall * L
+    ok = {k: o.double().cpu().numpy()[:, :cut] for k, o in zip(parity.OUTPUTS, out)}
+    parity.assert_parity(ok, {k: ref[k][:, :cut] for k in parity.OUTPUTS}, 1e-5, time_axis=1)
+    # the stalled chunk itself is NaN
+    assert np.isnan(lam[:, cut:cut + L]).all()
+    # a later chunk either composed the stalled chunk's published aggregate
+    # (decoupled look-back: exact) or read its poisoned inclusive state (NaN)
+    for c0 in range(cut + L, w.T, L):
+        blk = {k: o.double().cpu().numpy()[:, c0:c0 + L] for k, o in zip(parity.OUTPUTS, out)}
+        if np.isnan(blk["lam"]).all():
+            continue
+        assert np.isfinite(blk["lam"]).all()
+        parity.assert_parity(blk, {k: ref[k][:, c0:c0 + L] for k in parity.OUTPUTS}, 1e-5, time_axis=1)
+    # the context is still usable and a normal call is correct again
+    out2 = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out2)}
+    parity.assert_parity(got, ref, 1e-5, time_axis=1)

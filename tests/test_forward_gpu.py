@@ -1,0 +1,171 @@
+"""kla_scan_forward (CUDA, through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from kalman_linear_attention_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _kla():
+    import kalman_linear_attention_b200 as kla
+    return kla
+
+
+def _run_full(w, **kw):
+    """Device run + oracle over every channel (small shapes)."""
+    kla = _kla()
+    x = wl.generate(w)
+    dt = parity.torch_dtype(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV).to(dt) for k in wl.INPUT_NAMES}
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], torch.from_numpy(x["lam0"]).to(DEV),
+                           torch.from_numpy(x["eta0"]).to(DEV), **kw)
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {k: (None if o is None else o.double().cpu().numpy()) for k, o in zip(parity.OUTPUTS, out)}
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], threads=8)
+    return got, ref, x
+
+
+# (B, T, H, N): tile-aligned, ragged chunk tail, ragged channel tile, tiny and
+# odd shapes that take the plain-load path, long enough for deep look-back.
+SHAPES = [
+    (1, 256, 1, 64),     # the tiny workload's shape
+    (2, 200, 3, 40),     # HN = 120: ragged channel tile, ragged last chunk (TMA path)
+    (3, 130, 1, 7),      # HN = 7: plain-load path, ragged everything
+    (1, 1, 1, 1),        # one token, one channel
+    (2, 63, 2, 32),      # T shorter than a chunk
+    (1, 4099, 2, 64),    # 65 chunks: multi-hop look-back
+    (5, 96, 4, 16),      # B > 1 with a second chunk
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("family", ["tiny", "stiff", "lm_layer"])
+def test_parity_small_shapes(shape, family):
+    B, T, H, N = shape
+    w = wl.WORKLOADS[family].with_shape(B=B, T=T, H=H, N=N)
+    got, ref, _ = _run_full(w)
+    parity.assert_parity(got, ref, parity.RTOL[w.dtype], time_axis=1, what=f"{family} {shape}")
+
+
+def test_tiny_workload_exact_sizes():
+    w = wl.WORKLOADS["tiny"]
+    got, ref, _ = _run_full(w)
+    errs = parity.assert_parity(got, ref, parity.RTOL["f32"], time_axis=1, what="tiny")
+    print("tiny max errors", errs)
+
+
+def test_optional_outputs_skipped():
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=300, H=2, N=64)
+    full, ref, _ = _run_full(w)
+    part, _, _ = _run_full(w, want_mu=False, want_var=False)
+    assert part["mu"] is None and part["var"] is None
+    np.testing.assert_array_equal(full["lam"], part["lam"])
+    np.testing.assert_array_equal(full["eta"], part["eta"])
+
+
+def test_tma_and_plain_paths_agree():
+    """The same inputs through the TMA path (16-byte aligned) and the plain-load
+    path (inputs offset by one element) give bit-identical outputs."""
+    kla = _kla()
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=700, H=2, N=64)
+    x = wl.generate(w)
+    outs = []
+    for offset in (0, 1):
+        d = {}
+        for k in wl.INPUT_NAMES:
+            buf = torch.empty(x[k].size + offset, dtype=torch.float32, device=DEV)
+            d[k] = buf[offset:].view(x[k].shape)
+            d[k].copy_(torch.from_numpy(x[k]))
+        o = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], torch.from_numpy(x["lam0"]).to(DEV),
+                             torch.from_numpy(x["eta0"]).to(DEV))
+        outs.append([t.cpu() for t in o])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_workspace_contents_do_not_matter():
+    kla = _kla()
+    w = wl.WORKLOADS["stiff"].with_shape(B=3, T=500, H=2, N=64)
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
+    ws = kla.new_workspace(w.B, w.T, w.H, w.N, torch.float32, DEV)
+    results = []
+    for fill in (0x00, 0xFF, 0x5A):
+        ws.fill_(fill)
+        o = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"], workspace=ws)
+        results.append([t.clone() for t in o])
+    for r in results[1:]:
+        for a, b in zip(results[0], r):
+            assert torch.equal(a, b)
+
+
+def test_empty_problems():
+    kla = _kla()
+    for shape in ((0, 5, 1, 4), (1, 0, 1, 4), (1, 5, 0, 4)):
+        B, T, H, N = shape
+        z = torch.zeros(shape, device=DEV)
+        pri = torch.ones((B, H, N), device=DEV)
+        out = kla.scan_forward(z, z, z, z, pri, pri * 0)
+        assert out[0].shape == shape
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+
+
+def test_prefill_then_decode_continues_the_filter():
+    """The last row of a forward scan is the decode state: forward over T1,
+    then T2 decode steps, equals the oracle over T1 + T2 tokens."""
+    kla = _kla()
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=150, H=2, N=64)
+    x = wl.generate(w)
+    T1 = 100
+    d = {k: torch.from_numpy(np.ascontiguousarray(x[k])).to(DEV) for k in x}
+    lam, eta, _, _ = kla.scan_forward(*(d[k][:, :T1].contiguous() for k in wl.INPUT_NAMES),
+                                      d["lam0"], d["eta0"])
+    ls, es = lam[:, -1].contiguous(), eta[:, -1].contiguous()
+    mu = torch.empty_like(ls)
+    var = torch.empty_like(ls)
+    for t in range(T1, w.T):
+        kla.scan_step(*(d[k][:, t].contiguous() for k in wl.INPUT_NAMES), ls, es, mu_out=mu, var_out=var)
+    torch.cuda.synchronize()
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    got = {"lam": ls.double().cpu().numpy(), "eta": es.double().cpu().numpy(),
+           "mu": mu.double().cpu().numpy(), "var": var.double().cpu().numpy()}
+    last = {k: ref[k][:, -1] for k in parity.OUTPUTS}
+    # time axis is gone; scale eta / mu by the channel's rms over the whole sequence
+    rms = {k: np.sqrt(np.mean(ref[k] ** 2, axis=1)) for k in ("eta", "mu")}
+    for k in ("lam", "var"):
+        assert np.max(np.abs(got[k] - last[k]) / last[k]) <= 1e-5, k
+    for k in ("eta", "mu"):
+        assert np.max(np.abs(got[k] - last[k]) / (np.abs(last[k]) + rms[k])) <= 1e-5, k
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["tiny", "lm_layer", "long", "stiff"])
+def test_workload_full_size_sampled(name):
+    """Full-size workloads, launched exactly as the benchmark launches them;
+    the oracle checks a seeded sample of whole channels (every token)."""
+    kla = _kla()
+    w = wl.WORKLOADS[name]
+    sample = wl.channel_sample(w, 48)
+    d, sampled = parity.to_device(w, DEV, sample)
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    HN = w.H * w.N
+    got = {k: parity.gather_channels(o, sample, HN) for k, o in zip(parity.OUTPUTS, out)}
+    ref = parity.oracle_on_sample(sampled, np.ones(len(sample)), np.zeros(len(sample)))
+    errs = parity.assert_parity(got, ref, parity.RTOL[w.dtype], time_axis=0, what=name)
+    print(name, "max errors", errs)
+    # properties over every output element
+    lam = out[0]
+    assert bool(torch.isfinite(lam).all()) and bool((lam > 0).all())
+    assert bool(torch.isfinite(out[1]).all())
+    vl = out[3] * lam
+    assert float((vl - 1).abs().max()) < 1e-6
