@@ -32,6 +32,9 @@ constexpr int kL = 64;
 constexpr int kCW = 64;
 constexpr int kR = 4;
 constexpr int kNW = kCW / 32;
+// Checkpoint interval of the cross-chunk carry, in chunks (<= 32: one lane
+// of the look-back warp per flag).
+constexpr int kCkpt = 8;
 
 constexpr size_t kHeaderBytes = 256;  // ticket counter + padding
 constexpr int kMaxGrid = 0x7fffffff;
@@ -250,6 +253,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
     prm.flags = reinterpret_cast<unsigned *>(ws + lay.flags_off);
     prm.agg_ws = reinterpret_cast<float *>(ws + lay.agg_off);
     prm.incl_ws = reinterpret_cast<float *>(ws + lay.incl_off);
+    prm.ckpt = kCkpt;
     prm.wait_ns = g_wait_ns.load();
     prm.stall_chunk = g_stall_chunk.load();
 

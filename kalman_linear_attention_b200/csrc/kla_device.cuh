@@ -154,21 +154,26 @@ __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
 
-// Warp-wide bounded wait until *flag != 0.  Every lane of the warp must call
-// it.  Returns the flag value, or 0 when `limit_ns` ran out first.  The
-// iteration cap is a second bound in case the global timer misbehaves.
-__device__ __forceinline__ unsigned warp_wait_flag(const unsigned *flag, uint64_t limit_ns) {
+// Warp-wide bounded wait: every lane of the warp calls it with its own flag
+// pointer (or nullptr for "nothing to wait for"); returns true once every
+// lane's flag is nonzero, false when `limit_ns` ran out first.  The final
+// __syncwarp orders each lane's acquire before every lane's later loads.
+// The iteration cap is a second bound in case the global timer misbehaves.
+__device__ __forceinline__ bool warp_wait_flags(const unsigned *flag, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     unsigned ns = 32;
     for (uint32_t it = 0; it < (1u << 22); ++it) {
-        const unsigned v = ld_acquire_gpu(flag);
-        if (__all_sync(0xffffffffu, v != 0u)) return __shfl_sync(0xffffffffu, v, 0);
+        const unsigned v = flag != nullptr ? ld_acquire_gpu(flag) : 1u;
+        if (__all_sync(0xffffffffu, v != 0u)) {
+            __syncwarp();
+            return true;
+        }
         const bool late = (globaltimer_ns() - t0) > limit_ns;
-        if (__any_sync(0xffffffffu, late)) return 0u;
+        if (__any_sync(0xffffffffu, late)) return false;
         __nanosleep(ns);
         ns = ns < 1024 ? ns * 2 : 1024;
     }
-    return 0u;
+    return false;
 }
 
 // ---------------------------------------------------------------------------

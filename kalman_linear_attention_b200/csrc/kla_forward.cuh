@@ -13,10 +13,13 @@
 //   2. reduce   each thread folds its S tokens into a 3x3 homogeneous
 //               aggregate (see Agg in kla_device.cuh);
 //   3. carry    the first row of threads composes the R aggregates into the
-//               chunk aggregate, publishes it, and obtains the state entering
-//               the chunk by decoupled look-back over the preceding chunks of
-//               the same channels (aggregates of chunks still in flight are
-//               composed; the first finished chunk found ends the walk);
+//               chunk aggregate.  Every D-th chunk is a checkpoint: it
+//               publishes the state leaving it; every other chunk publishes
+//               its aggregate.  The state entering chunk c is the aggregates
+//               of chunks c-1 ... j+1 applied, in that fixed order, to the
+//               state leaving the last checkpoint j < c.  The serial chain is
+//               one hop per D chunks, and the result does not depend on
+//               timing (bitwise reproducible);
 //   4. filter   each thread enters its run with the state given by the carry
 //               and the aggregates of the runs before it, then runs the plain
 //               per-token recursion over its S tokens (exact up to fp32
@@ -24,8 +27,8 @@
 //               var into shared memory;
 //   5. store    the tile's outputs go back with TMA bulk-tensor stores.
 //
-// Every input and output byte crosses HBM once; the carries add 36 bytes
-// per channel per chunk.  Chunks are taken in ticket order from a global
+// Every input and output byte crosses HBM once; the carries add at most 28
+// bytes per channel per chunk (written once, read from L2).  Chunks are taken in ticket order from a global
 // counter, so a CTA only ever waits on CTAs that started before it, and
 // every wait is bounded (a timeout writes NaN and records an error).
 #pragma once
@@ -48,9 +51,10 @@ struct FwdParams {
     int nct;                       // channel tiles per batch row
     int nchunks;                   // chunks per sequence
     unsigned *ticket;              // global ticket counter (zeroed per call)
-    unsigned *flags;               // [tiles][CW / 32] : 0 empty, 1 aggregate, 2 inclusive
+    unsigned *flags;               // [tiles][CW / 32] : 0 empty, 1 aggregate, 2 carried state
+    int64_t ckpt;                  // checkpoint interval D in chunks (1 <= D <= 32)
     float *agg_ws;                 // [tiles][7][CW]
-    float *incl_ws;                // [tiles][2][CW]
+    float *incl_ws;                // [tiles][2][CW] (checkpoint chunks only)
     uint64_t wait_ns;              // bound of every wait
     int64_t stall_chunk;           // test hook: chunk whose look-back waits on never_set (-1: off)
 };
@@ -100,7 +104,7 @@ __device__ __forceinline__ Agg agg_load_l2(const float *base, int stride) {
 }
 
 template <typename Tin, int L, int CW, int R, bool TMA>
-__global__ void __launch_bounds__(CW * R, 2)
+__global__ void __launch_bounds__(CW * R, 3)
 kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
     using Cfg = FwdTile<Tin, L, CW, R>;
     constexpr int S = Cfg::S;
@@ -199,6 +203,8 @@ kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
             agg_renorm(tot);
         }
         unsigned *my_flag = prm.flags + tile * Cfg::NW + w;
+        const int64_t D = prm.ckpt;
+        const bool is_ckpt = (chunk % D) == 0;
         float lam_in, eta_in;
         if (load_failed) {
             lam_in = __int_as_float(0x7fc00000);
@@ -207,48 +213,38 @@ kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
             lam_in = valid ? prm.lam0[bb * prm.HN + ch] : 1.f;
             eta_in = valid ? prm.eta0[bb * prm.HN + ch] : 0.f;
         } else {
-            if (publish) {
-                float *dst = prm.agg_ws + tile * 7 * CW + c;
-                agg_store_smem(dst, CW, tot);
+            if (publish && !is_ckpt) {  // aggregate for the chunks up to the next checkpoint
+                agg_store_smem(prm.agg_ws + tile * 7 * CW + c, CW, tot);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) st_release_gpu(my_flag, 1u);
             }
-            // decoupled look-back over the chunks before this one
-            Agg acc = agg_identity();
-            bool have_acc = false;
-            int64_t j = tile - prm.tiles_per_chunk;
-            const unsigned *wait_on = (chunk == prm.stall_chunk) ? &g_never_set_word
-                                                                  : prm.flags + j * Cfg::NW + w;
-            for (;;) {
-                const unsigned st = warp_wait_flag(wait_on, prm.wait_ns);
-                if (st == 0u) {  // ran out of time: poison this chunk and everything after it
-                    lam_in = __int_as_float(0x7fc00000);
-                    eta_in = lam_in;
-                    if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
-                    break;
+            // Carry = (aggregates of chunks chunk-1 ... j+1) applied to the
+            // carried state of the checkpoint chunk j, in that fixed order.
+            const int64_t j = ((chunk - 1) / D) * D;
+            const int nd = (int)(chunk - j);  // chunks to read, <= D <= 32
+            const unsigned *f = lane < nd ? prm.flags + (tile - (int64_t)(lane + 1) * prm.tiles_per_chunk) * Cfg::NW + w
+                                          : nullptr;
+            if (chunk == prm.stall_chunk) f = lane == 0 ? &g_never_set_word : nullptr;
+            if (!warp_wait_flags(f, prm.wait_ns)) {  // ran out of time: poison this chunk
+                lam_in = __int_as_float(0x7fc00000);
+                eta_in = lam_in;
+                if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
+            } else {
+                Agg acc = agg_identity();
+                for (int i = 0; i + 1 < nd; ++i) {
+                    const int64_t jt = tile - (int64_t)(i + 1) * prm.tiles_per_chunk;
+                    const Agg g = agg_load_l2(prm.agg_ws + jt * 7 * CW + c, CW);
+                    acc = i == 0 ? g : agg_compose(acc, g);
+                    agg_renorm(acc);
                 }
-                if (st == 2u) {
-                    lam_in = __ldcg(prm.incl_ws + j * 2 * CW + c);
-                    eta_in = __ldcg(prm.incl_ws + j * 2 * CW + CW + c);
-                    if (have_acc) agg_apply(acc, lam_in, eta_in);
-                    break;
-                }
-                const Agg gj = agg_load_l2(prm.agg_ws + j * 7 * CW + c, CW);
-                acc = have_acc ? agg_compose(acc, gj) : gj;
-                agg_renorm(acc);
-                have_acc = true;
-                j -= prm.tiles_per_chunk;
-                if (j < 0) {  // unreachable: chunk 0 only ever publishes an inclusive state
-                    lam_in = __int_as_float(0x7fc00000);
-                    eta_in = lam_in;
-                    if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
-                    break;
-                }
-                wait_on = prm.flags + j * Cfg::NW + w;
+                const int64_t jt = tile - (int64_t)nd * prm.tiles_per_chunk;
+                lam_in = __ldcg(prm.incl_ws + jt * 2 * CW + c);
+                eta_in = __ldcg(prm.incl_ws + jt * 2 * CW + CW + c);
+                if (nd > 1) agg_apply(acc, lam_in, eta_in);
             }
         }
-        if (publish) {
+        if (publish && is_ckpt) {  // carried state out of a checkpoint chunk
             float li = lam_in, ei = eta_in;
             agg_apply(tot, li, ei);
             prm.incl_ws[tile * 2 * CW + c] = li;
@@ -329,8 +325,8 @@ __global__ void kla_clear_kernel(uint4 *p, int64_t n16) {
 
 // Test hook: a bounded wait on a flag nothing sets.
 __global__ void kla_unset_flag_wait_kernel(uint64_t wait_ns) {
-    const unsigned st = warp_wait_flag(&g_never_set_word, wait_ns);
-    if (st == 0u && threadIdx.x == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
+    const bool ok = warp_wait_flags(threadIdx.x == 0 ? &g_never_set_word : nullptr, wait_ns);
+    if (!ok && threadIdx.x == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
 }
 
 }  // namespace kla
