@@ -326,6 +326,8 @@ def run_ours(args):
     torch.cuda.set_device(device)
 
     base = wl.WORKLOADS[args.workload]
+    if args.tokens:
+        base = base.with_shape(T=args.tokens)
     w = rank_workload(base, rank)
     keep_host = not args.no_e2e
     dev, host = inputs_to_device(w, device, keep_host=keep_host)
@@ -437,6 +439,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long", choices=sorted(k for k, v in wl.WORKLOADS.items()
                                                                   if not v.decode))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (smaller cases for profiler captures; not a bench line)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--decode-replays", type=int, default=5)
     ap.add_argument("--ref-channels", type=int, default=256)
