@@ -75,7 +75,8 @@ typedef enum {
     KLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the required size */
     KLA_ERR_CUDA = 4,                /* a CUDA runtime / driver call failed */
     KLA_ERR_TIMEOUT = 5,             /* a device-side bounded wait ran out */
-    KLA_ERR_MISALIGNED = 6           /* workspace not 256-byte aligned */
+    KLA_ERR_MISALIGNED = 6,          /* workspace not 256-byte aligned */
+    KLA_ERR_TOO_LARGE = 7            /* problem exceeds the static scratch of kla_scan_forward_static */
 } kla_status_t;
 
 /* ABI version of the loaded library (KLA_ABI_VERSION it was built with). */
@@ -120,6 +121,44 @@ kla_status_t kla_scan_forward(const void *a, const void *p, const void *phi, con
                               float *lambda_out, float *eta_out, float *mu_out, float *var_out,
                               int64_t B, int64_t T, int64_t H, int64_t N,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Size of the static device scratch array used by kla_scan_forward_static. */
+#define KLA_STATIC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+
+/*
+ * kla_scan_forward for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot call cudaMalloc (or torch's allocator) at the point where they
+ * run the filter -- for example code running inside a CUDA stream capture,
+ * code under a fixed memory budget, or a host runtime without an allocator of
+ * its own -- and so cannot provide the workspace kla_scan_forward needs.
+ *
+ * Same arguments, results and errors as kla_scan_forward, minus the
+ * workspace: the carry scratch is a static device array of
+ * KLA_STATIC_SCRATCH_BYTES inside this library (one per device that loads
+ * the library, held until the process exits).  The call allocates and frees
+ * nothing.  The caller still provides the inputs and outputs.
+ *
+ * - Size limit: a problem is accepted when kla_scan_forward_workspace_size()
+ *   reports at most KLA_STATIC_SCRATCH_BYTES (about 59 million
+ *   token-channels with full 64-channel tiles, e.g. B=8, T=2048, H=16,
+ *   N=128); larger problems return KLA_ERR_TOO_LARGE before anything is
+ *   enqueued.
+ * - First call on a device: it looks up the device address of the static
+ *   array (cudaGetSymbolAddress) with that device current, and caches it.
+ *   Make that first call before any stream capture begins.
+ * - Sharing: every call on a device uses the same array, which keeps what the
+ *   last call left in it; each call re-zeroes, on its stream, the part that
+ *   must start at zero.  Calls whose work overlaps on the GPU (two streams,
+ *   two host threads) race on the array and give wrong results: serialise
+ *   them, or use kla_scan_forward with one workspace each.
+ */
+kla_status_t kla_scan_forward_static(const void *a, const void *p, const void *phi, const void *b,
+                                     kla_dtype_t in_dtype,
+                                     const float *lambda0, const float *eta0,
+                                     float *lambda_out, float *eta_out, float *mu_out, float *var_out,
+                                     int64_t B, int64_t T, int64_t H, int64_t N, void *stream);
 
 /*
  * One recurrent decode token for every channel (constant work per token;

@@ -20,9 +20,11 @@ KLA_F32 = 0
 KLA_BF16 = 1
 STATUS = {0: "KLA_OK", 1: "KLA_ERR_INVALID_ARG", 2: "KLA_ERR_UNSUPPORTED_DTYPE",
           3: "KLA_ERR_WORKSPACE_TOO_SMALL", 4: "KLA_ERR_CUDA", 5: "KLA_ERR_TIMEOUT",
-          6: "KLA_ERR_MISALIGNED"}
+          6: "KLA_ERR_MISALIGNED", 7: "KLA_ERR_TOO_LARGE"}
 KLA_OK, KLA_ERR_INVALID_ARG, KLA_ERR_UNSUPPORTED_DTYPE = 0, 1, 2
 KLA_ERR_WORKSPACE_TOO_SMALL, KLA_ERR_CUDA, KLA_ERR_TIMEOUT, KLA_ERR_MISALIGNED = 3, 4, 5, 6
+KLA_ERR_TOO_LARGE = 7
+STATIC_SCRATCH_BYTES = 32 << 20  # KLA_STATIC_SCRATCH_BYTES
 
 # Every exported symbol of include/kla.h, with (restype, argtypes).
 _VP, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -40,6 +42,8 @@ SIGNATURES = {
     "kla_debug_unset_flag_wait": (ctypes.c_int, [_VP]),
     "kla_forward_chunk_tokens": (ctypes.c_int, []),
     "kla_debug_stall_chunk": (ctypes.c_int, [_I64]),
+    "kla_scan_forward_static": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
+                                               _VP, _VP, _I64, _I64, _I64, _I64, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -231,3 +235,27 @@ def debug_unset_flag_wait(stream: Optional[torch.cuda.Stream] = None) -> None:
 
 def debug_stall_chunk(chunk: int) -> None:
     _check(lib().kla_debug_stall_chunk(int(chunk)), "kla_debug_stall_chunk")
+
+
+def scan_forward_static(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.Tensor,
+                        lam0: torch.Tensor, eta0: torch.Tensor,
+                        out: Sequence[Optional[torch.Tensor]],
+                        stream: Optional[torch.cuda.Stream] = None) -> None:
+    """kla_scan_forward_static: the forward scan for callers that cannot
+    allocate device memory.  The caller passes every tensor, outputs
+    included (``out`` = lambda, eta, mu, var; mu / var may be None); the
+    library uses its own fixed static device scratch (KLA_STATIC_SCRATCH_BYTES),
+    so nothing is allocated.  Calls that overlap on the GPU share that scratch
+    and must be serialised.  Raises KlaError(KLA_ERR_TOO_LARGE) when the
+    problem does not fit."""
+    if not (a.shape == p.shape == phi.shape == b.shape) or a.dim() != 4:
+        raise ValueError("a, p, phi, b must share one [B, T, H, N] shape")
+    B, T, H, N = a.shape
+    outs = list(out)
+    _require_cuda(a, p, phi, b, lam0, eta0, *outs)
+    with torch.cuda.device(a.device):
+        st = lib().kla_scan_forward_static(
+            _ptr(a), _ptr(p), _ptr(phi), _ptr(b), _dtype_code(a), _ptr(lam0), _ptr(eta0),
+            _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), B, T, H, N,
+            _stream_handle(stream))
+    _check(st, "kla_scan_forward_static")

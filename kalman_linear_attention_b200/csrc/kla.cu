@@ -188,6 +188,9 @@ KLA_API const char *kla_strerror(kla_status_t s) {
         case KLA_ERR_CUDA: return "KLA_ERR_CUDA: a CUDA call failed";
         case KLA_ERR_TIMEOUT: return "KLA_ERR_TIMEOUT: a device-side bounded wait ran out";
         case KLA_ERR_MISALIGNED: return "KLA_ERR_MISALIGNED: workspace must be 256-byte aligned";
+        case KLA_ERR_TOO_LARGE:
+            return "KLA_ERR_TOO_LARGE: the problem needs more scratch than the library's static array "
+                   "(KLA_STATIC_SCRATCH_BYTES); use kla_scan_forward with a caller-allocated workspace";
     }
     return "unknown kla_status_t";
 }
@@ -360,4 +363,62 @@ KLA_API kla_status_t kla_debug_stall_chunk(int64_t chunk) {
     if (chunk < -1) return KLA_ERR_INVALID_ARG;
     g_stall_chunk.store(chunk);
     return KLA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// kla_scan_forward_static: kla_scan_forward without a caller-provided
+// workspace, for callers that cannot allocate device memory.
+//
+// The carry scratch is this file-scope device array, KLA_STATIC_SCRATCH_BYTES
+// long.  Every device that loads the library holds one copy of it until the
+// process exits.  Host code cannot use the array's name as a device address
+// (in host code it names a host-side shadow), so the device address is looked
+// up once per device with cudaGetSymbolAddress, with that device current, on
+// the first call made on it, and cached.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_scratch[KLA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 256;
+
+// Device address of g_static_scratch on the current device (nullptr on error).
+void *static_scratch_address() {
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+KLA_API kla_status_t kla_scan_forward_static(const void *a, const void *p, const void *phi,
+                                             const void *b, kla_dtype_t in_dtype,
+                                             const float *lambda0, const float *eta0,
+                                             float *lambda_out, float *eta_out, float *mu_out,
+                                             float *var_out, int64_t B, int64_t T, int64_t H,
+                                             int64_t N, void *stream) {
+    size_t need = 0;
+    const kla_status_t st = kla_scan_forward_workspace_size(B, T, H, N, in_dtype, &need);
+    if (st != KLA_OK) return st;
+    if (need > (size_t)KLA_STATIC_SCRATCH_BYTES) return KLA_ERR_TOO_LARGE;
+    if (need == 0)  // empty problem: validate and return without touching the device
+        return kla_scan_forward(a, p, phi, b, in_dtype, lambda0, eta0, lambda_out, eta_out, mu_out,
+                                var_out, B, T, H, N, nullptr, 0, stream);
+    void *scratch = static_scratch_address();
+    if (scratch == nullptr) return KLA_ERR_CUDA;
+    // kla_scan_forward zeroes the part of the scratch that must start at zero
+    // (ticket counter and ready flags) on `stream` before its scan kernel.
+    return kla_scan_forward(a, p, phi, b, in_dtype, lambda0, eta0, lambda_out, eta_out, mu_out,
+                            var_out, B, T, H, N, scratch, (size_t)KLA_STATIC_SCRATCH_BYTES, stream);
 }

@@ -38,7 +38,7 @@ def test_abi_version(lib):
 
 
 def test_strerror(lib):
-    for code in range(7):
+    for code in range(8):
         assert lib.kla_strerror(code)
     assert b"unknown" in lib.kla_strerror(99)
 
