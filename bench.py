@@ -91,15 +91,15 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel: int):
     """DRAM bytes per launch from a committed ncu summary, only if it was
-    taken on the kernel sources as they are now."""
+    taken on this kernel with the kernel sources as they are now."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("kernel_sha") != kernel_source_hash():
+    if not e or e.get("kernel_sha") != kernel_source_hash() or e.get("kernel") != kernel:
         return None
     return float(e["dram_bytes_per_launch"])
 
@@ -194,6 +194,7 @@ def time_forward(kla, w, dev, steps: int, warmup: int, dist_mod):
     outs = [torch.empty((B, T, H, N), dtype=torch.float32, device=dev["a"].device) for _ in range(4)]
     ws = kla.new_workspace(B, T, H, N, dev["a"].dtype, dev["a"].device)
     stream = torch.cuda.current_stream()
+    plan = kla.forward_plan(dev["a"], dev["p"], dev["phi"], dev["b"])
     args = (dev["a"], dev["p"], dev["phi"], dev["b"], dev["lam0"], dev["eta0"])
     for _ in range(warmup):
         kla.scan_forward(*args, out=outs, workspace=ws)
@@ -218,7 +219,7 @@ def time_forward(kla, w, dev, steps: int, warmup: int, dist_mod):
         raise RuntimeError("device-side error in the timed region")
     total_ms = t_start.elapsed_time(t_end)
     per_launch = [a.elapsed_time(b) for a, b in ev]
-    return total_ms, per_launch
+    return total_ms, per_launch, plan
 
 
 def time_e2e(kla, w, host, steps: int):
@@ -334,7 +335,10 @@ def run_ours(args):
 
     sampler = ClockSampler(local)
     sampler.start()
-    total_ms, per_launch = time_forward(kla, w, dev, args.steps, args.warmup, dist if world > 1 else None)
+    total_ms, per_launch, plan = time_forward(kla, w, dev, args.steps, args.warmup,
+                                              dist if world > 1 else None)
+    kernel_name = {1: "kla_forward_kernel (chunked; + its workspace clear kernel, timed together)",
+                   2: "kla_forward_stream_kernel (channel-owning streaming)"}[plan[0]]
     clocks = sampler.stop()
 
     max_ms = max_over_ranks(total_ms, dist if world > 1 else None)
@@ -345,7 +349,8 @@ def run_ours(args):
     launch_ms = statistics.mean(per_launch)
     achieved = bpt * tc_rank / (launch_ms * 1e-3) / 1e9
     peak, peak_src = measured_peaks()
-    traffic = recorded_traffic(args.workload)
+    traffic = recorded_traffic(args.workload if not args.tokens else f"{args.workload}@T={args.tokens}",
+                               plan[0])
 
     e2e = None
     if host is not None:
@@ -384,9 +389,8 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
                      "traffic": traffic, "algorithmic_bytes_per_launch": bpt * tc_rank,
-                     "kernel": "kla_forward_kernel (+ its workspace clear, timed together)",
-                     "launch_ms": launch_ms},
-        "gpu_launches": 2 * args.steps,
+                     "kernel": kernel_name, "launch_ms": launch_ms},
+        "gpu_launches": plan[1] * args.steps,
         "clocks": clocks,
         "e2e": e2e,
         "decode": decode,

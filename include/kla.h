@@ -122,6 +122,31 @@ kla_status_t kla_scan_forward(const void *a, const void *p, const void *phi, con
                               int64_t B, int64_t T, int64_t H, int64_t N,
                               void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Which forward kernel kla_scan_forward would launch for a problem of this
+ * shape and dtype with these input pointers (only their alignment matters;
+ * they are not dereferenced), written to *kernel: 1 = the chunked kernel whose
+ * chunks exchange carries through the workspace, 2 = the channel-owning
+ * streaming kernel; *launches = the kernel launches one call enqueues (2 and
+ * 1 respectively: the chunked kernel is preceded by a workspace clear).
+ * 0 and 0 for an empty problem.  Honours kla_debug_force_forward_kernel.
+ */
+kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
+                                   const void *a, const void *p, const void *phi, const void *b,
+                                   int *kernel, int *launches);
+
+/*
+ * Test hook: which forward kernel kla_scan_forward calls enqueued afterwards
+ * use.  0 (default): chosen by shape; 1: the chunked kernel whose chunks
+ * exchange carries through the workspace (any shape); 2: the channel-owning
+ * streaming kernel (used only when its geometry holds: 16-byte aligned
+ * inputs, H*N*elem a multiple of 16 bytes, H*N >= 32, T >= 32; otherwise the
+ * chunked kernel runs).  Both compute the same filter; their chunkings differ,
+ * so results agree to rounding, not bit for bit.  KLA_ERR_INVALID_ARG for
+ * other values.
+ */
+kla_status_t kla_debug_force_forward_kernel(int which);
+
 /* Size of the static device scratch array used by kla_scan_forward_static. */
 #define KLA_STATIC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
 

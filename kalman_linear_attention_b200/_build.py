@@ -11,8 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(HERE, "libkla.so")
 SOURCES = [os.path.join(CSRC, "kla.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("kla_device.cuh", "kla_forward.cuh", "kla_step.cuh")] \
-    + [os.path.join(INCLUDE, "kla.h")]
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "kla.h")]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17",

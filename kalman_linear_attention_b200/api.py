@@ -42,6 +42,9 @@ SIGNATURES = {
     "kla_debug_unset_flag_wait": (ctypes.c_int, [_VP]),
     "kla_forward_chunk_tokens": (ctypes.c_int, []),
     "kla_debug_stall_chunk": (ctypes.c_int, [_I64]),
+    "kla_debug_force_forward_kernel": (ctypes.c_int, [ctypes.c_int]),
+    "kla_scan_forward_plan": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP, _VP, _VP,
+                                             ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "kla_scan_forward_static": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
                                                _VP, _VP, _I64, _I64, _I64, _I64, _VP]),
 }
@@ -112,6 +115,18 @@ def workspace_size(B: int, T: int, H: int, N: int, dtype: torch.dtype = torch.fl
     _check(lib().kla_scan_forward_workspace_size(B, T, H, N, code, ctypes.byref(out)),
            "kla_scan_forward_workspace_size")
     return int(out.value)
+
+
+def forward_plan(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.Tensor) -> Tuple[int, int]:
+    """(kernel, launches) that scan_forward would use for these inputs:
+    kernel 1 = chunked (workspace carries), 2 = channel-owning streaming."""
+    B, T, H, N = a.shape
+    k, n = ctypes.c_int(0), ctypes.c_int(0)
+    with torch.cuda.device(a.device):
+        _check(lib().kla_scan_forward_plan(B, T, H, N, _dtype_code(a), _ptr(a), _ptr(p), _ptr(phi),
+                                           _ptr(b), ctypes.byref(k), ctypes.byref(n)),
+               "kla_scan_forward_plan")
+    return int(k.value), int(n.value)
 
 
 def chunk_tokens() -> int:
@@ -231,6 +246,11 @@ def set_wait_limit_ns(ns: int) -> None:
 
 def debug_unset_flag_wait(stream: Optional[torch.cuda.Stream] = None) -> None:
     _check(lib().kla_debug_unset_flag_wait(_stream_handle(stream)), "kla_debug_unset_flag_wait")
+
+
+def debug_force_forward_kernel(which: int) -> None:
+    """0: choose by shape; 1: chunked kernel (workspace carries); 2: streaming kernel."""
+    _check(lib().kla_debug_force_forward_kernel(int(which)), "kla_debug_force_forward_kernel")
 
 
 def debug_stall_chunk(chunk: int) -> None:

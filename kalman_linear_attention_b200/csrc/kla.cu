@@ -16,6 +16,7 @@
 #include <utility>
 
 #include "kla_forward.cuh"
+#include "kla_forward_stream.cuh"
 #include "kla_step.cuh"
 
 #define KLA_API extern "C" __attribute__((visibility("default")))
@@ -28,13 +29,51 @@ using kla::StepParams;
 
 // Tile geometry of the forward scan: L tokens x CW channels per CTA, R rows
 // of threads (S = L / R tokens per thread).
-constexpr int kL = 64;
-constexpr int kCW = 64;
-constexpr int kR = 4;
+// (Overridable at build time for tuning sweeps.)
+#ifndef KLA_TILE_L
+#define KLA_TILE_L 64
+#endif
+#ifndef KLA_TILE_CW
+#define KLA_TILE_CW 64
+#endif
+#ifndef KLA_TILE_R
+#define KLA_TILE_R 4
+#endif
+#ifndef KLA_CKPT
+#define KLA_CKPT 8
+#endif
+constexpr int kL = KLA_TILE_L;
+constexpr int kCW = KLA_TILE_CW;
+constexpr int kR = KLA_TILE_R;
 constexpr int kNW = kCW / 32;
 // Checkpoint interval of the cross-chunk carry, in chunks (<= 32: one lane
 // of the look-back warp per flag).
-constexpr int kCkpt = 8;
+constexpr int kCkpt = KLA_CKPT;
+static_assert(kCkpt >= 1 && kCkpt <= 32, "checkpoint interval must be 1..32");
+
+// Channel-owning streaming kernel: chunk length, chunk warps, ring stages.
+// The chunk warps hold a whole chunk in registers (4 x L floats per thread).
+// 11 chunk warps + the producer = 12 warps = 3 per SM sub-partition, which
+// allows 168 registers per thread (enough for L = 32 without spills).
+#ifndef KLA_STREAM_L
+#define KLA_STREAM_L 32
+#endif
+#ifndef KLA_STREAM_W
+#define KLA_STREAM_W 11
+#endif
+#ifndef KLA_STREAM_SMEM
+#define KLA_STREAM_SMEM (200 * 1024)
+#endif
+constexpr int kSL = KLA_STREAM_L;
+constexpr int kSW = KLA_STREAM_W;
+template <typename Tin>
+constexpr int stream_stages() {
+    return (KLA_STREAM_SMEM - 4096) / (4 * kSL * 32 * (int)sizeof(Tin));
+}
+
+// 0: choose by shape; 1: the chunked kernel with cross-CTA carries; 2: the
+// channel-owning streaming kernel (test hook kla_debug_force_forward_kernel).
+std::atomic<int> g_force_kernel{0};
 
 constexpr size_t kHeaderBytes = 256;  // ticket counter + padding
 constexpr int kMaxGrid = 0x7fffffff;
@@ -166,6 +205,64 @@ cudaError_t launch_forward(const FwdParams &prm, const FwdMaps &maps, int64_t ti
     return cudaGetLastError();
 }
 
+int sm_count() {
+    static std::mutex mu;
+    static int count[256] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        count[dev] = n;
+    }
+    return count[dev];
+}
+
+template <typename Tin>
+cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &maps, cudaStream_t stream) {
+    constexpr int NS = stream_stages<Tin>();
+    using Cfg = kla::StreamTile<Tin, kSL, kSW, NS>;
+    static_assert(NS >= 2 && Cfg::SMEM <= 227 * 1024, "stream kernel shared memory");
+    auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, kSW, NS>;
+    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(prm.ntiles, sm_count());
+    kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    return cudaGetLastError();
+}
+
+// [B, T, HN] tensor viewed as dims {HN, T, B}, box {32, kSL, 1}.
+bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz,
+                       int64_t B, int64_t T, int64_t HN) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)HN, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)(HN * esz), (cuuint64_t)(T * HN * esz)};
+    const cuuint32_t box[3] = {32u, (cuuint32_t)kSL, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2: the channel-owning streaming kernel -- its TMA geometry holds (16-byte
+//    aligned inputs, H*N*elem a multiple of 16 bytes, H*N >= 32, T >= one
+//    chunk) and there are at least 0.8 x (SM count) tiles of 32 channels to
+//    keep the GPU busy, or the test hook forces it;
+// 1: the chunked kernel with cross-CTA carries (any shape).
+int forward_kernel_choice(int64_t B, int64_t T, int64_t HN, size_t esz, const void *a, const void *p,
+                          const void *phi, const void *b) {
+    const int force = g_force_kernel.load();
+    if (force == 1) return 1;
+    const bool geometry = (HN * (int64_t)esz) % 16 == 0 && T >= kSL && HN >= 32 && aligned16(a) &&
+                          aligned16(p) && aligned16(phi) && aligned16(b) && encode_fn() != nullptr;
+    if (!geometry) return 1;
+    if (force == 2) return 2;
+    const int64_t ntiles32 = B * ((HN + 31) / 32);
+    return ntiles32 * 5 >= (int64_t)sm_count() * 4 ? 2 : 1;
+}
+
 cudaError_t launch_clear(void *ws, size_t bytes, cudaStream_t stream) {
     const int64_t n16 = (int64_t)(bytes / 16);
     const int threads = 256;
@@ -260,6 +357,32 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
     prm.wait_ns = g_wait_ns.load();
     prm.stall_chunk = g_stall_chunk.load();
 
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const CUtensorMapDataType tdt =
+        in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+
+    // The channel-owning streaming kernel when forward_kernel_choice picks it
+    // (it needs no workspace); otherwise the chunked kernel below.
+    if (forward_kernel_choice(B, T, HN, esz, a, p, phi, b) == 2) {
+        FwdMaps smaps;
+        std::memset(&smaps, 0, sizeof(smaps));
+        const void *ins4[4] = {a, p, phi, b};
+        bool ok = true;
+        for (int k = 0; k < 4 && ok; ++k) ok = encode_stream_map(&smaps.in[k], ins4[k], tdt, esz, B, T, HN);
+        if (ok) {
+            kla::StreamParams sp;
+            sp.lam0 = lambda0; sp.eta0 = eta0;
+            sp.out[0] = lambda_out; sp.out[1] = eta_out; sp.out[2] = mu_out; sp.out[3] = var_out;
+            sp.T = T; sp.HN = HN; sp.ntiles = B * ((HN + 31) / 32);
+            sp.nct = (int)((HN + 31) / 32);
+            sp.nchunks = (int)((T + kSL - 1) / kSL);
+            sp.wait_ns = g_wait_ns.load();
+            const cudaError_t es = in_dtype == KLA_F32 ? launch_forward_stream<float>(sp, smaps, st)
+                                                       : launch_forward_stream<__nv_bfloat16>(sp, smaps, st);
+            return es == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+        }
+    }
+
     // TMA boxes when the geometry allows them; plain loads otherwise.
     FwdMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -268,15 +391,12 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
     for (int k = 0; k < 8 && tma; ++k)
         if (ptrs[k] && !aligned16(ptrs[k])) tma = false;
     if (tma) {
-        const CUtensorMapDataType dt =
-            in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-        for (int k = 0; k < 4 && tma; ++k) tma = encode_map(&maps.in[k], ptrs[k], dt, esz, B, T, HN);
+        for (int k = 0; k < 4 && tma; ++k) tma = encode_map(&maps.in[k], ptrs[k], tdt, esz, B, T, HN);
         for (int k = 0; k < 4 && tma; ++k)
             if (ptrs[4 + k])
                 tma = encode_map(&maps.out[k], ptrs[4 + k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN);
     }
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (launch_clear(ws, lay.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
     cudaError_t e;
     if (in_dtype == KLA_F32)
@@ -358,6 +478,29 @@ KLA_API kla_status_t kla_debug_unset_flag_wait(void *stream) {
 }
 
 KLA_API int kla_forward_chunk_tokens(void) { return kL; }
+
+KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
+                                           const void *a, const void *p, const void *phi, const void *b,
+                                           int *kernel, int *launches) {
+    if (!kernel || !launches || B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems)) return KLA_ERR_INVALID_ARG;
+    if (elems == 0) {
+        *kernel = 0;
+        *launches = 0;
+        return KLA_OK;
+    }
+    *kernel = forward_kernel_choice(B, T, HN, dtype_size(in_dtype), a, p, phi, b);
+    *launches = *kernel == 2 ? 1 : 2;
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_debug_force_forward_kernel(int which) {
+    if (which < 0 || which > 2) return KLA_ERR_INVALID_ARG;
+    g_force_kernel.store(which);
+    return KLA_OK;
+}
 
 KLA_API kla_status_t kla_debug_stall_chunk(int64_t chunk) {
     if (chunk < -1) return KLA_ERR_INVALID_ARG;

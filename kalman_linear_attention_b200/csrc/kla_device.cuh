@@ -59,8 +59,12 @@ __device__ __forceinline__ Agg agg_identity() {
 }
 
 // Rescale by 2^-e so that the largest Moebius entry lies in [1, 2).  A
-// multiplication by a power of two is exact, so the represented map is
-// unchanged.
+// multiplication by a power of two is exact, so the represented map -- and
+// every later rounding -- is unchanged: how often this runs does not change
+// any result bit (barring overflow).  The kernels run it every second token;
+// between two runs the largest entry grows at most by the square of the
+// largest row sum of M_t, so entries stay finite while
+// 1 + p phi + a^2 phi + p + a^2 < 2^63 per token.
 __device__ __forceinline__ void agg_renorm(Agg &g) {
     const float mx = fmaxf(fmaxf(fabsf(g.m11), fabsf(g.m12)), fmaxf(fabsf(g.m21), fabsf(g.m22)));
     int e = (__float_as_int(mx) >> 23) & 0xff;  // biased exponent of the max
@@ -98,12 +102,23 @@ __device__ __forceinline__ Agg agg_compose(const Agg &X, const Agg &Y) {
     return r;
 }
 
+// Hardware reciprocal (PTX rcp.approx.ftz.f32, one MUFU instruction; the PTX
+// ISA bounds its error by 1 ulp for normal inputs).  The filter's state is
+// positive and far from the subnormal range under the documented
+// preconditions, and its error per token is damped by the contraction of the
+// recursion, so this keeps the results well inside the parity tolerance.
+__device__ __forceinline__ float rcp_hw(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // State (lambda, eta) after the span of g, entered with (lam, eta).
 __device__ __forceinline__ void agg_apply(const Agg &g, float &lam, float &eta) {
     const float n = fmaf(g.m11, lam, g.m12);
     const float d = fmaf(g.m21, lam, g.m22);
     const float h = fmaf(g.g1, lam, fmaf(g.A, eta, g.g2));
-    const float rd = 1.f / d;
+    const float rd = rcp_hw(d);
     lam = n * rd;
     eta = h * rd;
 }
@@ -117,10 +132,10 @@ struct TokenOut { float lam, eta, mu, var; };
 __device__ __forceinline__ TokenOut filter_token(float &lam, float &eta,
                                                  float a, float p, float phi, float b) {
     const float den = fmaf(p, lam, a * a);
-    const float r = 1.f / den;           // IEEE round-to-nearest reciprocal
+    const float r = rcp_hw(den);
     lam = fmaf(lam, r, phi);
     eta = fmaf(a * r, eta, b);
-    const float v = 1.f / lam;
+    const float v = rcp_hw(lam);
     TokenOut o;
     o.lam = lam; o.eta = eta; o.mu = eta * v; o.var = v;
     return o;
@@ -159,6 +174,9 @@ __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
 // lane's flag is nonzero, false when `limit_ns` ran out first.  The final
 // __syncwarp orders each lane's acquire before every lane's later loads.
 // The iteration cap is a second bound in case the global timer misbehaves.
+#ifndef KLA_SPIN_NS_MAX
+#define KLA_SPIN_NS_MAX 1024
+#endif
 __device__ __forceinline__ bool warp_wait_flags(const unsigned *flag, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     unsigned ns = 32;
@@ -171,7 +189,7 @@ __device__ __forceinline__ bool warp_wait_flags(const unsigned *flag, uint64_t l
         const bool late = (globaltimer_ns() - t0) > limit_ns;
         if (__any_sync(0xffffffffu, late)) return false;
         __nanosleep(ns);
-        ns = ns < 1024 ? ns * 2 : 1024;
+        ns = ns < KLA_SPIN_NS_MAX ? ns * 2 : KLA_SPIN_NS_MAX;
     }
     return false;
 }

@@ -103,8 +103,12 @@ __device__ __forceinline__ Agg agg_load_l2(const float *base, int stride) {
     return g;
 }
 
+#ifndef KLA_MIN_BLOCKS
+#define KLA_MIN_BLOCKS 3
+#endif
+
 template <typename Tin, int L, int CW, int R, bool TMA>
-__global__ void __launch_bounds__(CW * R, 3)
+__global__ void __launch_bounds__(CW * R, KLA_MIN_BLOCKS)
 kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
     using Cfg = FwdTile<Tin, L, CW, R>;
     constexpr int S = Cfg::S;
@@ -182,9 +186,10 @@ kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
                 const int i = t * CW + c;
                 agg_push_token(g, to_f32(s_in[i]), to_f32(s_in[LC + i]),
                                to_f32(s_in[2 * LC + i]), to_f32(s_in[3 * LC + i]));
-                agg_renorm(g);
+                if (s & 1) agg_renorm(g);
             }
         }
+        agg_renorm(g);
         agg_store_smem(s_agg + r * 7 * CW + c, CW, g);
     }
     __syncthreads();

@@ -92,3 +92,21 @@ def test_host_argument_errors(lib):
     assert step(*sargs(B=0)) == 0
     assert lib.kla_set_wait_limit_ns(0) == 1
     assert lib.kla_debug_stall_chunk(-5) == 1
+
+
+def test_forward_plan_host_decision(lib):
+    """The plan query answers on the host: empty problems launch nothing, and
+    inputs the streaming kernel cannot take (unaligned, narrow, short) go to
+    the chunked kernel (2 launches: workspace clear + scan)."""
+    k, n = ctypes.c_int(-1), ctypes.c_int(-1)
+    A = 1 << 20
+    assert lib.kla_scan_forward_plan(1, 0, 32, 128, 0, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) == (0, 0)
+    assert lib.kla_scan_forward_plan(1, 65536, 32, 128, 0, A + 4, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) == (1, 2)                      # unaligned input
+    assert lib.kla_scan_forward_plan(1, 65536, 1, 7, 0, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) == (1, 2)                      # H*N = 7
+    assert lib.kla_scan_forward_plan(1, 65536, 32, 128, 0, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) in ((1, 2), (2, 1))           # 2 needs a driver for TMA maps
+    assert lib.kla_scan_forward_plan(-1, 1, 1, 1, 0, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 1
+    assert lib.kla_scan_forward_plan(1, 1, 1, 1, 5, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 2

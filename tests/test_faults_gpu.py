@@ -17,7 +17,9 @@ DEV = "cuda:0"
 def kla():
     import kalman_linear_attention_b200 as kla
     kla.set_wait_limit_ns(2_000_000)  # 2 ms
+    kla.debug_force_forward_kernel(1)  # the kernel whose chunks wait on each other across CTAs
     yield kla
+    kla.debug_force_forward_kernel(0)
     kla.debug_stall_chunk(-1)
     kla.set_wait_limit_ns(1_000_000_000)
 

@@ -17,6 +17,16 @@ def _kla():
     return kla
 
 
+@pytest.fixture(params=[1, 2], ids=["chunked", "stream"])
+def kernel(request):
+    """Force one of the two forward kernels (1: chunks exchange carries through
+    the workspace; 2: channel-owning streaming kernel, where its geometry holds)."""
+    kla = _kla()
+    kla.debug_force_forward_kernel(request.param)
+    yield request.param
+    kla.debug_force_forward_kernel(0)
+
+
 def _run_full(w, **kw):
     """Device run + oracle over every channel (small shapes)."""
     kla = _kla()
@@ -47,21 +57,21 @@ SHAPES = [
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("family", ["tiny", "stiff", "lm_layer"])
-def test_parity_small_shapes(shape, family):
+def test_parity_small_shapes(shape, family, kernel):
     B, T, H, N = shape
     w = wl.WORKLOADS[family].with_shape(B=B, T=T, H=H, N=N)
     got, ref, _ = _run_full(w)
     parity.assert_parity(got, ref, parity.RTOL[w.dtype], time_axis=1, what=f"{family} {shape}")
 
 
-def test_tiny_workload_exact_sizes():
+def test_tiny_workload_exact_sizes(kernel):
     w = wl.WORKLOADS["tiny"]
     got, ref, _ = _run_full(w)
     errs = parity.assert_parity(got, ref, parity.RTOL["f32"], time_axis=1, what="tiny")
     print("tiny max errors", errs)
 
 
-def test_optional_outputs_skipped():
+def test_optional_outputs_skipped(kernel):
     w = wl.WORKLOADS["tiny"].with_shape(B=2, T=300, H=2, N=64)
     full, ref, _ = _run_full(w)
     part, _, _ = _run_full(w, want_mu=False, want_var=False)
@@ -71,9 +81,11 @@ def test_optional_outputs_skipped():
 
 
 def test_tma_and_plain_paths_agree():
-    """The same inputs through the TMA path (16-byte aligned) and the plain-load
-    path (inputs offset by one element) give bit-identical outputs."""
+    """The same inputs through the chunked kernel's TMA path (16-byte aligned)
+    and its plain-load path (inputs offset by one element) give bit-identical
+    outputs."""
     kla = _kla()
+    kla.debug_force_forward_kernel(1)
     w = wl.WORKLOADS["tiny"].with_shape(B=2, T=700, H=2, N=64)
     x = wl.generate(w)
     outs = []
@@ -86,11 +98,28 @@ def test_tma_and_plain_paths_agree():
         o = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], torch.from_numpy(x["lam0"]).to(DEV),
                              torch.from_numpy(x["eta0"]).to(DEV))
         outs.append([t.cpu() for t in o])
+    kla.debug_force_forward_kernel(0)
     for a, b in zip(*outs):
         assert torch.equal(a, b)
 
 
-def test_workspace_contents_do_not_matter():
+def test_kernels_agree_to_rounding():
+    """The two forward kernels chunk the scan differently; their outputs agree
+    within the fp32 tolerance (and each matches the oracle elsewhere)."""
+    kla = _kla()
+    w = wl.WORKLOADS["stiff"].with_shape(B=8, T=3000, H=2, N=64)
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
+    res = []
+    for which in (1, 2):
+        kla.debug_force_forward_kernel(which)
+        o = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+        res.append({k: t.double().cpu().numpy() for k, t in zip(parity.OUTPUTS, o)})
+    kla.debug_force_forward_kernel(0)
+    parity.assert_parity(res[1], res[0], 2e-6, time_axis=1, what="stream vs chunked")
+
+
+def test_workspace_contents_do_not_matter(kernel):
     kla = _kla()
     w = wl.WORKLOADS["stiff"].with_shape(B=3, T=500, H=2, N=64)
     x = wl.generate(w)
@@ -118,7 +147,7 @@ def test_empty_problems():
     assert kla.get_error() == 0
 
 
-def test_prefill_then_decode_continues_the_filter():
+def test_prefill_then_decode_continues_the_filter(kernel):
     """The last row of a forward scan is the decode state: forward over T1,
     then T2 decode steps, equals the oracle over T1 + T2 tokens."""
     kla = _kla()
@@ -149,29 +178,38 @@ def test_prefill_then_decode_continues_the_filter():
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["tiny", "lm_layer", "long", "stiff"])
 def test_workload_full_size_sampled(name):
-    """Full-size workloads, launched exactly as the benchmark launches them;
-    the oracle checks a seeded sample of whole channels (every token)."""
+    """Full-size workloads, launched exactly as the benchmark launches them
+    (default kernel choice), then with each forward kernel forced; the oracle
+    checks a seeded sample of whole channels (every token)."""
     kla = _kla()
     w = wl.WORKLOADS[name]
     sample = wl.channel_sample(w, 48)
     d, sampled = parity.to_device(w, DEV, sample)
-    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
-    torch.cuda.synchronize()
-    assert kla.get_error() == 0
-    HN = w.H * w.N
-    got = {k: parity.gather_channels(o, sample, HN) for k, o in zip(parity.OUTPUTS, out)}
     ref = parity.oracle_on_sample(sampled, np.ones(len(sample)), np.zeros(len(sample)))
-    errs = parity.assert_parity(got, ref, parity.RTOL[w.dtype], time_axis=0, what=name)
-    print(name, "max errors", errs)
-    # properties over every output element
-    lam = out[0]
-    assert bool(torch.isfinite(lam).all()) and bool((lam > 0).all())
-    assert bool(torch.isfinite(out[1]).all())
-    vl = out[3] * lam
-    assert float((vl - 1).abs().max()) < 1e-6
+    HN = w.H * w.N
+    try:
+        for which in (0, 1, 2):
+            kla.debug_force_forward_kernel(which)
+            out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+            torch.cuda.synchronize()
+            assert kla.get_error() == 0
+            got = {k: parity.gather_channels(o, sample, HN) for k, o in zip(parity.OUTPUTS, out)}
+            errs = parity.assert_parity(got, ref, parity.RTOL[w.dtype], time_axis=0,
+                                        what=f"{name} kernel={which}")
+            print(name, "kernel", which, "max errors", errs)
+            # properties over every output element
+            lam = out[0]
+            assert bool(torch.isfinite(lam).all()) and bool((lam > 0).all())
+            assert bool(torch.isfinite(out[1]).all())
+            vl = out[3] * lam
+            assert float((vl - 1).abs().max()) < 1e-6
+            del out, lam, vl
+            torch.cuda.empty_cache()
+    finally:
+        kla.debug_force_forward_kernel(0)
 
 
-def test_bitwise_reproducible():
+def test_bitwise_reproducible(kernel):
     """The carry is composed in a fixed order, so repeated calls agree bit for bit."""
     kla = _kla()
     w = wl.WORKLOADS["tiny"].with_shape(B=2, T=6000, H=4, N=64)
@@ -182,3 +220,15 @@ def test_bitwise_reproducible():
         again = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
         for a, b in zip(first, again):
             assert torch.equal(a, b)
+
+
+def test_plan_matches_workloads():
+    """On a B200 the standard workloads take the streaming kernel except the
+    tiny one (2 tiles of 32 channels cannot occupy the GPU)."""
+    kla = _kla()
+    for name, expect in (("tiny", 1), ("lm_layer", 2), ("long", 2), ("stiff", 2)):
+        w = wl.WORKLOADS[name]
+        dt = parity.torch_dtype(w)
+        z = torch.empty((w.B, w.T, w.H, w.N), dtype=dt, device=DEV)
+        assert kla.forward_plan(z, z, z, z)[0] == expect, name
+        del z
