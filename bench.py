@@ -360,8 +360,9 @@ def run_ours(args):
         e2e_s = max_over_ranks(e2e_s, dist if world > 1 else None)
         e2e = {"value": tc_all / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_s * 1e3,
-               "how": "scan_forward on pinned host tensors: H2D of a, p, phi, b, lam0, eta0, "
-                      "the scan, D2H of lambda, eta, mu, var, stream sync; wall clock"}
+               "how": "scan_forward on pinned host tensors (C ABI kla_scan_forward_host): the sequence in "
+                      "8 blocks, H2D of a, p, phi, b (+ lam0, eta0), scan, D2H of lambda, eta, mu, var "
+                      "pipelined on three streams, then a stream sync; wall clock"}
     decode = None
     if not args.no_decode:
         decode = time_decode(kla, device, None, args.decode_replays)

@@ -186,6 +186,41 @@ kla_status_t kla_scan_forward_static(const void *a, const void *p, const void *p
                                      int64_t B, int64_t T, int64_t H, int64_t N, void *stream);
 
 /*
+ * Device workspace that kla_scan_forward_host needs (two device slots of one
+ * block each, plus the scan workspace of one block), written to *bytes.
+ * t_block = tokens per block, or 0 to let the library pick (about T / 8,
+ * whole 64-token chunks).
+ */
+kla_status_t kla_scan_forward_host_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                                  kla_dtype_t in_dtype, int64_t t_block, size_t *bytes);
+
+/*
+ * The forward filter on HOST buffers (same arguments and results as
+ * kla_scan_forward, but a, p, phi, b, lambda0, eta0 and the outputs are host
+ * memory, ideally page-locked).  The sequence is processed in blocks of
+ * t_block tokens: the copy of block k+1 to the device, the scan of block k
+ * (entering with the state that left block k-1, i.e. its last lambda / eta
+ * row) and the copy of block k-1 back overlap on two internal copy streams and
+ * `stream`.  Sequences longer than device memory can thus be filtered.
+ *
+ *   workspace   device memory of at least
+ *               kla_scan_forward_host_workspace_size(...) bytes, 256-byte
+ *               aligned, owned by the caller.
+ *   stream      the caller's stream; when it reaches the end of the call every
+ *               output has been written to host memory.
+ *
+ * The internal copy streams and events are created once per device; calls on
+ * one device must not overlap (serialise them on one stream).  Results agree
+ * with kla_scan_forward to rounding (block boundaries are extra carry points).
+ */
+kla_status_t kla_scan_forward_host(const void *a, const void *p, const void *phi, const void *b,
+                                   kla_dtype_t in_dtype,
+                                   const float *lambda0, const float *eta0,
+                                   float *lambda_out, float *eta_out, float *mu_out, float *var_out,
+                                   int64_t B, int64_t T, int64_t H, int64_t N, int64_t t_block,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent decode token for every channel (constant work per token;
  * the running posterior is a sufficient summary: "Kalman filter" primer
  * section 6.2, and the review's O(1)-per-step recurrent form).

@@ -9,7 +9,7 @@ torch nor the built library.
 _API_NAMES = {
     "scan_forward", "scan_step", "workspace_size", "new_workspace", "get_error",
     "set_wait_limit_ns", "debug_unset_flag_wait", "debug_stall_chunk", "chunk_tokens",
-    "debug_force_forward_kernel", "forward_plan",
+    "debug_force_forward_kernel", "forward_plan", "host_workspace_size",
     "KlaError", "lib", "load_library", "scan_forward_static",
 }
 

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(HERE, "libkla.so")
-SOURCES = [os.path.join(CSRC, "kla.cu")]
+SOURCES = [os.path.join(CSRC, "kla.cu"), os.path.join(CSRC, "kla_host.cu")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "kla.h")]
 
 NVCC_FLAGS = [

@@ -47,6 +47,10 @@ SIGNATURES = {
                                              ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "kla_scan_forward_static": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP,
                                                _VP, _VP, _I64, _I64, _I64, _I64, _VP]),
+    "kla_scan_forward_host_workspace_size": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int, _I64,
+                                                            ctypes.POINTER(_SZ)]),
+    "kla_scan_forward_host": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP,
+                                             _I64, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -166,24 +170,8 @@ def scan_forward(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.T
         raise TypeError("lam0 and eta0 must be float32")
     host = not a.is_cuda
     if host:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        nb = a.is_pinned()
-        s = stream if stream is not None else torch.cuda.current_stream(dev)
-        with torch.cuda.stream(s):
-            d_in = [x.to(dev, non_blocking=nb) for x in (a, p, phi, b, lam0, eta0)]
-            d_out = scan_forward(*d_in, want_mu=want_mu, want_var=want_var, stream=s,
-                                 workspace=workspace)
-            res = []
-            for i, d in enumerate(d_out):
-                if d is None:
-                    res.append(None)
-                    continue
-                dst = out[i] if out is not None and out[i] is not None else \
-                    torch.empty(d.shape, dtype=d.dtype, pin_memory=nb)
-                dst.copy_(d, non_blocking=nb)
-                res.append(dst)
-        s.synchronize()
-        return tuple(res)
+        return _scan_forward_host(a, p, phi, b, lam0, eta0, want_mu=want_mu, want_var=want_var, out=out,
+                                  workspace=workspace, stream=stream)
 
     _require_cuda(a, p, phi, b, lam0, eta0)
     code = _dtype_code(a)
@@ -202,6 +190,47 @@ def scan_forward(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.T
         st = kla_scan_forward_raw(a, p, phi, b, code, lam0, eta0, outs, B, T, H, N, workspace,
                                   _stream_handle(stream))
     _check(st, "kla_scan_forward")
+    return tuple(outs)
+
+
+def host_workspace_size(B: int, T: int, H: int, N: int, dtype: torch.dtype = torch.float32,
+                        t_block: int = 0) -> int:
+    code = KLA_BF16 if dtype == torch.bfloat16 else KLA_F32
+    out = ctypes.c_size_t(0)
+    _check(lib().kla_scan_forward_host_workspace_size(B, T, H, N, code, t_block, ctypes.byref(out)),
+           "kla_scan_forward_host_workspace_size")
+    return int(out.value)
+
+
+def _scan_forward_host(a, p, phi, b, lam0, eta0, *, want_mu, want_var, out, workspace, stream,
+                       t_block: int = 0):
+    """kla_scan_forward_host: host tensors in and out, copies pipelined with
+    the scan on the current CUDA device; returns after the outputs are in
+    host memory."""
+    for t in (a, p, phi, b, lam0, eta0):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host path: every tensor must be a contiguous CPU tensor")
+    B, T, H, N = a.shape
+    pinned = a.is_pinned()
+    if out is None:
+        outs = [torch.empty((B, T, H, N), dtype=torch.float32, pin_memory=pinned),
+                torch.empty((B, T, H, N), dtype=torch.float32, pin_memory=pinned),
+                torch.empty((B, T, H, N), dtype=torch.float32, pin_memory=pinned) if want_mu else None,
+                torch.empty((B, T, H, N), dtype=torch.float32, pin_memory=pinned) if want_var else None]
+    else:
+        outs = list(out)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if workspace is None:
+        workspace = torch.empty(max(host_workspace_size(B, T, H, N, a.dtype, t_block), 1), dtype=torch.uint8,
+                                device=dev)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        st = lib().kla_scan_forward_host(
+            _ptr(a), _ptr(p), _ptr(phi), _ptr(b), _dtype_code(a), _ptr(lam0), _ptr(eta0),
+            _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), B, T, H, N, t_block,
+            _ptr(workspace), workspace.numel(), s.cuda_stream)
+    _check(st, "kla_scan_forward_host")
+    s.synchronize()
     return tuple(outs)
 
 

@@ -51,24 +51,45 @@ constexpr int kNW = kCW / 32;
 constexpr int kCkpt = KLA_CKPT;
 static_assert(kCkpt >= 1 && kCkpt <= 32, "checkpoint interval must be 1..32");
 
-// Channel-owning streaming kernel: chunk length, chunk warps, ring stages.
-// The chunk warps hold a whole chunk in registers (4 x L floats per thread).
-// 11 chunk warps + the producer = 12 warps = 3 per SM sub-partition, which
-// allows 168 registers per thread (enough for L = 32 without spills).
+// Channel-owning streaming kernel: chunk length, chunk warps, output group,
+// ring stages.  The chunk warps hold a whole chunk in registers (4 x L floats
+// per thread); up to 12 warps = 3 per SM sub-partition allow 168 registers
+// per thread.
 #ifndef KLA_STREAM_L
 #define KLA_STREAM_L 32
 #endif
-#ifndef KLA_STREAM_W
-#define KLA_STREAM_W 11
+// Chunk warps: fp32 stages are 16 KB, so 9 warps leave two ring stages free
+// for prefetch; bf16 stages are 8 KB and the ring is deep anyway, so 11
+// (12 warps in all = 3 per SM sub-partition, the most that still allows 168
+// registers per thread).
+#ifndef KLA_STREAM_W_F32
+#define KLA_STREAM_W_F32 9
+#endif
+#ifndef KLA_STREAM_W_BF16
+#define KLA_STREAM_W_BF16 11
+#endif
+#ifndef KLA_STREAM_G
+#define KLA_STREAM_G 4
 #endif
 #ifndef KLA_STREAM_SMEM
-#define KLA_STREAM_SMEM (200 * 1024)
+#define KLA_STREAM_SMEM (227 * 1024)
+#endif
+#ifndef KLA_STREAM_MAX_STAGES
+#define KLA_STREAM_MAX_STAGES 24
 #endif
 constexpr int kSL = KLA_STREAM_L;
-constexpr int kSW = KLA_STREAM_W;
+constexpr int kSG = KLA_STREAM_G;
+template <typename Tin> constexpr int stream_warps() {
+    return sizeof(Tin) == 4 ? KLA_STREAM_W_F32 : KLA_STREAM_W_BF16;
+}
+// Ring stages that fit beside the per-warp output buffers and carry slots.
 template <typename Tin>
 constexpr int stream_stages() {
-    return (KLA_STREAM_SMEM - 4096) / (4 * kSL * 32 * (int)sizeof(Tin));
+    constexpr int W = stream_warps<Tin>();
+    const int stage = 4 * kSL * 32 * (int)sizeof(Tin);
+    const int fixed = W * 2 * 4 * kSG * 32 * 4 + W * 2 * 32 * 4 + W * 8 + 2048;
+    const int ns = (KLA_STREAM_SMEM - fixed) / stage;
+    return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
 }
 
 // 0: choose by shape; 1: the chunked kernel with cross-CTA carries; 2: the
@@ -221,10 +242,11 @@ int sm_count() {
 
 template <typename Tin>
 cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &maps, cudaStream_t stream) {
+    constexpr int W = stream_warps<Tin>();
     constexpr int NS = stream_stages<Tin>();
-    using Cfg = kla::StreamTile<Tin, kSL, kSW, NS>;
+    using Cfg = kla::StreamTile<Tin, kSL, W, NS, kSG>;
     static_assert(NS >= 2 && Cfg::SMEM <= 227 * 1024, "stream kernel shared memory");
-    auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, kSW, NS>;
+    auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, W, NS, kSG>;
     cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(prm.ntiles, sm_count());
@@ -232,14 +254,14 @@ cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &m
     return cudaGetLastError();
 }
 
-// [B, T, HN] tensor viewed as dims {HN, T, B}, box {32, kSL, 1}.
+// [B, T, HN] tensor viewed as dims {HN, T, B}, box {32, rows, 1}.
 bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz,
-                       int64_t B, int64_t T, int64_t HN) {
+                       int64_t B, int64_t T, int64_t HN, int rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)HN, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[2] = {(cuuint64_t)(HN * esz), (cuuint64_t)(T * HN * esz)};
-    const cuuint32_t box[3] = {32u, (cuuint32_t)kSL, 1u};
+    const cuuint32_t box[3] = {32u, (cuuint32_t)rows, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -247,16 +269,18 @@ bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt,
 }
 
 // 2: the channel-owning streaming kernel -- its TMA geometry holds (16-byte
-//    aligned inputs, H*N*elem a multiple of 16 bytes, H*N >= 32, T >= one
-//    chunk) and there are at least 0.8 x (SM count) tiles of 32 channels to
-//    keep the GPU busy, or the test hook forces it;
+//    aligned inputs and outputs, H*N*elem a multiple of 16 bytes, H*N >= 32,
+//    T >= one chunk) and there are at least 0.8 x (SM count) tiles of 32
+//    channels to keep the GPU busy, or the test hook forces it;
 // 1: the chunked kernel with cross-CTA carries (any shape).
 int forward_kernel_choice(int64_t B, int64_t T, int64_t HN, size_t esz, const void *a, const void *p,
-                          const void *phi, const void *b) {
+                          const void *phi, const void *b, const void *o0, const void *o1, const void *o2,
+                          const void *o3) {
     const int force = g_force_kernel.load();
     if (force == 1) return 1;
     const bool geometry = (HN * (int64_t)esz) % 16 == 0 && T >= kSL && HN >= 32 && aligned16(a) &&
-                          aligned16(p) && aligned16(phi) && aligned16(b) && encode_fn() != nullptr;
+                          aligned16(p) && aligned16(phi) && aligned16(b) && aligned16(o0) && aligned16(o1) &&
+                          aligned16(o2) && aligned16(o3) && encode_fn() != nullptr;
     if (!geometry) return 1;
     if (force == 2) return 2;
     const int64_t ntiles32 = B * ((HN + 31) / 32);
@@ -363,16 +387,19 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
 
     // The channel-owning streaming kernel when forward_kernel_choice picks it
     // (it needs no workspace); otherwise the chunked kernel below.
-    if (forward_kernel_choice(B, T, HN, esz, a, p, phi, b) == 2) {
+    if (forward_kernel_choice(B, T, HN, esz, a, p, phi, b, lambda_out, eta_out, mu_out, var_out) == 2) {
         FwdMaps smaps;
         std::memset(&smaps, 0, sizeof(smaps));
         const void *ins4[4] = {a, p, phi, b};
         bool ok = true;
-        for (int k = 0; k < 4 && ok; ++k) ok = encode_stream_map(&smaps.in[k], ins4[k], tdt, esz, B, T, HN);
+        for (int k = 0; k < 4 && ok; ++k) ok = encode_stream_map(&smaps.in[k], ins4[k], tdt, esz, B, T, HN, kSL);
+        float *outs4[4] = {lambda_out, eta_out, mu_out, var_out};
+        for (int k = 0; k < 4 && ok; ++k)
+            if (outs4[k]) ok = encode_stream_map(&smaps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN, kSG);
         if (ok) {
             kla::StreamParams sp;
             sp.lam0 = lambda0; sp.eta0 = eta0;
-            sp.out[0] = lambda_out; sp.out[1] = eta_out; sp.out[2] = mu_out; sp.out[3] = var_out;
+            sp.write_mu = mu_out != nullptr; sp.write_var = var_out != nullptr;
             sp.T = T; sp.HN = HN; sp.ntiles = B * ((HN + 31) / 32);
             sp.nct = (int)((HN + 31) / 32);
             sp.nchunks = (int)((T + kSL - 1) / kSL);
@@ -491,7 +518,9 @@ KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int6
         *launches = 0;
         return KLA_OK;
     }
-    *kernel = forward_kernel_choice(B, T, HN, dtype_size(in_dtype), a, p, phi, b);
+    // outputs come from the caching allocator (aligned); only the inputs are passed here
+    *kernel = forward_kernel_choice(B, T, HN, dtype_size(in_dtype), a, p, phi, b, nullptr, nullptr, nullptr,
+                                    nullptr);
     *launches = *kernel == 2 ? 1 : 2;
     return KLA_OK;
 }

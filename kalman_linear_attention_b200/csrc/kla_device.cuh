@@ -75,18 +75,22 @@ __device__ __forceinline__ void agg_renorm(Agg &g) {
 }
 
 // g <- G_t * g : append one token (a, p, phi, b) after the span g covers.
+// M_t factors as [[1, phi], [0, 1]] * [[1, 0], [p, a^2]]: the predict step
+// (the denominator row becomes p n + a^2 d) followed by the update step (the
+// numerator row gains phi times the new denominator row) -- the matrix form
+// of "prior precision, then add the token's evidence precision".  Six
+// multiply-adds instead of ten, all on non-negative numbers.
 __device__ __forceinline__ void agg_push_token(Agg &g, float a, float p, float phi, float b) {
     const float a2 = a * a;
-    const float al = fmaf(p, phi, 1.f);  // 1 + p phi
-    const float be = a2 * phi;           // a^2 phi
-    const float n1 = fmaf(al, g.m11, be * g.m21);
-    const float n2 = fmaf(al, g.m12, be * g.m22);
-    const float d1 = fmaf(p, g.m11, a2 * g.m21);
+    const float d1 = fmaf(p, g.m11, a2 * g.m21);   // predict: denominator row
     const float d2 = fmaf(p, g.m12, a2 * g.m22);
-    g.g1 = fmaf(b, d1, a * g.g1);
+    g.m11 = fmaf(phi, d1, g.m11);                  // update: numerator row
+    g.m12 = fmaf(phi, d2, g.m12);
+    g.m21 = d1;
+    g.m22 = d2;
+    g.g1 = fmaf(b, d1, a * g.g1);                  // information row
     g.g2 = fmaf(b, d2, a * g.g2);
     g.A *= a;
-    g.m11 = n1; g.m12 = n2; g.m21 = d1; g.m22 = d2;
 }
 
 // X * Y : the span of Y followed by the span of X.

@@ -12,15 +12,19 @@
 //   W chunk warps   warp w takes chunks w, w + W, w + 2W, ...  Lane = channel.
 //                   A warp copies its chunk into registers and releases the
 //                   stage at once (so nearly the whole ring is in flight),
-//                   then (1) folds the L tokens into the
-//                   chunk's 3x3 homogeneous aggregate (no dependency on any
-//                   other chunk), (2) waits for the state leaving the previous
-//                   chunk (a shared-memory slot written by the previous warp,
-//                   mbarrier carry[slot]), applies its aggregate to it and
-//                   hands the result to the next warp -- the only serial link,
-//                   a few hundred cycles per chunk -- and (3) runs the plain
-//                   per-token recursion from the entering state, storing
-//                   lambda, eta, mu, var straight to global memory.
+//                   then (1) folds the L tokens into the chunk's 3x3
+//                   homogeneous aggregate (no dependency on any other chunk),
+//                   (2) waits for the state leaving the previous chunk (a
+//                   shared-memory slot written by the previous warp, mbarrier
+//                   carry[slot]), applies its aggregate to it and hands the
+//                   result to the next warp -- the only serial link, a few
+//                   hundred cycles per chunk -- and (3) runs the plain
+//                   per-token recursion from the entering state.  Outputs go
+//                   through a per-warp, double-buffered shared-memory box of
+//                   G tokens x 32 channels x 4 outputs and leave with TMA
+//                   bulk-tensor stores issued by the warp's lane 0 (which
+//                   also clip ragged edges), so the chunk warps do no global
+//                   address arithmetic.
 //
 // No global flags, fences or look-back: the W warps overlap their passes
 // while the producer keeps HBM busy.  Chunk aggregates are formed and applied
@@ -38,17 +42,28 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
 
+// Wait until at most N committed bulk store groups are still reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
+}
+
+// Wait until every committed bulk store group has completed (writes done).
+__device__ __forceinline__ void bulk_wait_group_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 struct StreamParams {
     const float *lam0, *eta0;      // [B, H, N] prior
-    float *out[4];                 // lambda, eta, mu, var ; mu / var may be null
     int64_t T, HN;
     int64_t ntiles;                // B * ceil(HN / 32)
     int nct;                       // 32-channel tiles per batch row
     int nchunks;                   // ceil(T / L)
+    int write_mu, write_var;       // outputs 2 / 3 requested
     uint64_t wait_ns;
 };
 
-template <typename Tin, int L, int W, int NS>
+template <typename Tin, int L, int W, int NS, int G>
 struct StreamTile {
     // Chunk j sits in stage j % NS and is handled by warp j % W.  With
     // NS >= W a warp waiting for stage s is always waiting for the stage's
@@ -56,10 +71,14 @@ struct StreamTile {
     // chunk, through the carry chain), so the parity of the mbarrier wait is
     // unambiguous.  With NS < W a warp could pass a wait one phase early.
     static_assert(NS >= W, "the stage ring must be at least as deep as the number of chunk warps");
+    static_assert(L % G == 0, "output groups must tile the chunk");
     static constexpr int CW = 32;
-    static constexpr int THREADS = 32 * (W + 1);
+    static constexpr int THREADS = 32 * (W + 1);                     // producer + W chunk warps
     static constexpr int STAGE_BYTES = 4 * L * CW * (int)sizeof(Tin);
-    static constexpr int CARRY_OFF = NS * STAGE_BYTES;                       // [W][2][32] fp32
+    static constexpr int OUTBOX_BYTES = G * CW * 4;                 // one output, one group
+    static constexpr int OUTBUF_BYTES = 4 * OUTBOX_BYTES;           // four outputs
+    static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][32] fp32
+    static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][32] fp32
     static constexpr int BAR_OFF = align_up(CARRY_OFF + W * 2 * CW * 4, 128);  // full, empty, carry
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
@@ -71,10 +90,10 @@ __device__ __forceinline__ void mbar_wait_or_flag(uint64_t *bar, unsigned parity
     }
 }
 
-template <typename Tin, int L, int W, int NS>
+template <typename Tin, int L, int W, int NS, int G>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
 kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMaps maps) {
-    using Cfg = StreamTile<Tin, L, W, NS>;
+    using Cfg = StreamTile<Tin, L, W, NS, G>;
     constexpr int LC = L * 32;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::BAR_OFF);
@@ -122,6 +141,8 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 
     // ------------------------------------------------------------ chunk warps
     const int w = warp - 1;
+    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
+    int group_seq = 0;  // output groups this warp has committed (bulk groups are per thread: lane 0)
 #pragma unroll 1
     for (int64_t j = w; j < my_chunks; j += W) {
         const int s = (int)(j % NS);
@@ -138,37 +159,56 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 
         // State entering chunk j (from the previous chunk's warp, or the prior
         // at a tile's first chunk); hands the state leaving it to the next warp.
-        auto chunk_carry = [&](int64_t jj, int64_t ck, const Agg &g, float &lam, float &eta) {
-            if (jj > 0) {
-                const int ps = (int)((jj - 1) % W);
-                mbar_wait_or_flag(&carry_bar[ps], (unsigned)(((jj - 1) / W) & 1), prm.wait_ns);
+        auto chunk_carry = [&](const Agg &g, float &lam, float &eta) {
+            if (j > 0) {
+                const int ps = (int)((j - 1) % W);
+                mbar_wait_or_flag(&carry_bar[ps], (unsigned)(((j - 1) / W) & 1), prm.wait_ns);
                 lam = slots[ps * 64 + lane];
                 eta = slots[ps * 64 + 32 + lane];
             }
-            if (ck == 0) {
+            if (chunk == 0) {
                 lam = cvalid ? prm.lam0[bb * prm.HN + ch] : 1.f;
                 eta = cvalid ? prm.eta0[bb * prm.HN + ch] : 0.f;
             }
             float lo = lam, eo = eta;
             agg_apply(g, lo, eo);
-            const int ms = (int)(jj % W);
+            const int ms = (int)(j % W);
             slots[ms * 64 + lane] = lo;
             slots[ms * 64 + 32 + lane] = eo;
             __syncwarp();
             if (lane == 0) mbar_arrive(&carry_bar[ms]);
         };
-        const int64_t gi = (bb * prm.T + t0) * prm.HN + ch;
-        float *o0 = prm.out[0] + gi, *o1 = prm.out[1] + gi;
-        float *o2 = prm.out[2] != nullptr ? prm.out[2] + gi : nullptr;
-        float *o3 = prm.out[3] != nullptr ? prm.out[3] + gi : nullptr;
-        const int64_t HN = prm.HN;
-        auto emit = [&](int t, const TokenOut &o) {
-            if (cvalid) {
-                __stcs(o0 + t * HN, o.lam);
-                __stcs(o1 + t * HN, o.eta);
-                if (o2 != nullptr) __stcs(o2 + t * HN, o.mu);
-                if (o3 != nullptr) __stcs(o3 + t * HN, o.var);
+
+        // Output group q of this chunk (tokens q*G .. q*G+G-1): claim a free
+        // half of the warp's double buffer (the store that last read it must
+        // be done), fill it, and send it out with TMA bulk-tensor stores.
+        auto group_begin = [&]() -> float * {
+            float *buf = outbuf0 + (group_seq & 1) * (Cfg::OUTBUF_BYTES / 4);
+            if (group_seq >= 2) {
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
             }
+            return buf;
+        };
+        auto group_end = [&](float *buf, int q) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int ty = (int)(t0 + q * G);
+                const int x = (int)(ct * 32);
+                tma_store_3d(&maps.out[0], buf, x, ty, (int)bb);
+                tma_store_3d(&maps.out[1], buf + G * 32, x, ty, (int)bb);
+                if (prm.write_mu) tma_store_3d(&maps.out[2], buf + 2 * G * 32, x, ty, (int)bb);
+                if (prm.write_var) tma_store_3d(&maps.out[3], buf + 3 * G * 32, x, ty, (int)bb);
+                bulk_commit_group();
+            }
+            ++group_seq;
+        };
+        auto put = [&](float *buf, int u, const TokenOut &o) {
+            buf[u * 32 + lane] = o.lam;
+            buf[G * 32 + u * 32 + lane] = o.eta;
+            buf[2 * G * 32 + u * 32 + lane] = o.mu;
+            buf[3 * G * 32 + u * 32 + lane] = o.var;
         };
 
         if (t_valid == L) {
@@ -196,15 +236,21 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             agg_renorm(g);
             // (2) carry
             float lam, eta;
-            chunk_carry(j, chunk, g, lam, eta);
+            chunk_carry(g, lam, eta);
             // (3) per-token recursion from the entering state
 #pragma unroll
-            for (int t = 0; t < L; ++t) {
-                const TokenOut o = filter_token(lam, eta, xa[t], xp[t], xf[t], xb[t]);
-                emit(t, o);
+            for (int q = 0; q < L / G; ++q) {
+                float *buf = group_begin();
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    const int t = q * G + u;
+                    put(buf, u, filter_token(lam, eta, xa[t], xp[t], xf[t], xb[t]));
+                }
+                group_end(buf, q);
             }
         } else {
-            // Ragged last chunk: straight from shared memory, released at the end.
+            // Ragged last chunk: straight from shared memory, released at the
+            // end; rows past T are clipped by the TMA stores.
             Agg g = agg_identity();
 #pragma unroll 2
             for (int t = 0; t < t_valid; ++t) {
@@ -215,18 +261,29 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             }
             agg_renorm(g);
             float lam, eta;
-            chunk_carry(j, chunk, g, lam, eta);
-#pragma unroll 2
-            for (int t = 0; t < t_valid; ++t) {
-                const int i = t * 32 + lane;
-                const TokenOut o = filter_token(lam, eta, to_f32(stage[i]), to_f32(stage[LC + i]),
-                                                to_f32(stage[2 * LC + i]), to_f32(stage[3 * LC + i]));
-                emit(t, o);
+            chunk_carry(g, lam, eta);
+            const int ngroups = (t_valid + G - 1) / G;
+#pragma unroll 1
+            for (int q = 0; q < ngroups; ++q) {
+                float *buf = group_begin();
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    const int t = q * G + u;
+                    if (t < t_valid) {
+                        const int i = t * 32 + lane;
+                        put(buf, u, filter_token(lam, eta, to_f32(stage[i]), to_f32(stage[LC + i]),
+                                                 to_f32(stage[2 * LC + i]), to_f32(stage[3 * LC + i])));
+                    }
+                }
+                group_end(buf, q);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
+    // every bulk store of this warp must be complete before the CTA exits
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
 }
 
 }  // namespace kla

@@ -110,3 +110,14 @@ def test_forward_plan_host_decision(lib):
     assert (k.value, n.value) in ((1, 2), (2, 1))           # 2 needs a driver for TMA maps
     assert lib.kla_scan_forward_plan(-1, 1, 1, 1, 0, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 1
     assert lib.kla_scan_forward_plan(1, 1, 1, 1, 5, A, A, A, A, ctypes.byref(k), ctypes.byref(n)) == 2
+
+
+def test_host_workspace_size(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.kla_scan_forward_host_workspace_size(1, 65536, 32, 128, 0, 0, ctypes.byref(out)) == 0
+    # about 8 blocks: 2 slots x one block x (16 + 16 bytes per token-channel) + one scan workspace
+    block = 8192 * 4096
+    assert 2 * block * 32 <= out.value <= 2 * block * 32 * 1.1
+    assert lib.kla_scan_forward_host_workspace_size(1, 0, 1, 1, 0, 0, ctypes.byref(out)) == 0 and out.value == 0
+    assert lib.kla_scan_forward_host_workspace_size(1, 10, 1, 1, 0, -1, ctypes.byref(out)) == 1
+    assert lib.kla_scan_forward_host_workspace_size(1, 10, 1, 1, 4, 0, ctypes.byref(out)) == 2

@@ -232,3 +232,67 @@ def test_plan_matches_workloads():
         z = torch.empty((w.B, w.T, w.H, w.N), dtype=dt, device=DEV)
         assert kla.forward_plan(z, z, z, z)[0] == expect, name
         del z
+
+
+def _special_inputs(kind, B=2, T=400, H=2, N=48, seed=77):
+    """Degenerate and special cases of the method, seeded."""
+    rng = np.random.default_rng(seed)
+    sh = (B, T, H, N)
+    a = rng.uniform(0.5, 1.0, sh)
+    p = np.exp(rng.uniform(np.log(1e-3), 0.0, sh))
+    phi = np.exp(rng.uniform(np.log(1e-2), np.log(10.0), sh))
+    b = rng.standard_normal(sh)
+    if kind == "no_process_noise":      # p = 0: the affine Moebius case
+        p[:] = 0.0
+        a = rng.uniform(0.98, 1.02, sh) * np.where(rng.random(sh) < 0.3, -1.0, 1.0)
+    elif kind == "no_observation":      # phi = 0, b = 0: every update leaves the prior
+        phi[:] = 0.0
+        b[:] = 0.0
+    elif kind == "precision_sum":       # a = 1, p = 0: lambda is a running sum of phi
+        a[:] = 1.0
+        p[:] = 0.0
+    elif kind == "negative_decay":      # the gate follows the sign of a
+        a *= np.where(rng.random(sh) < 0.5, -1.0, 1.0)
+    elif kind == "mixed_zeros":         # some tokens without noise, some without evidence
+        p[rng.random(sh) < 0.3] = 0.0
+        z = rng.random(sh) < 0.3
+        phi[z] = 0.0
+        b[z] = 0.0
+    x = {k: v.astype(np.float32) for k, v in (("a", a), ("p", p), ("phi", phi), ("b", b))}
+    x["lam0"] = rng.uniform(0.5, 2.0, (B, H, N)).astype(np.float32)
+    x["eta0"] = rng.standard_normal((B, H, N)).astype(np.float32)
+    return x
+
+
+SPECIAL = ["no_process_noise", "no_observation", "precision_sum", "negative_decay", "mixed_zeros"]
+
+
+@pytest.mark.parametrize("kind", SPECIAL)
+def test_special_cases_forward(kind, kernel):
+    kla = _kla()
+    x = _special_inputs(kind)
+    d = {k: torch.from_numpy(v).to(DEV) for k, v in x.items()}
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out)}
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    parity.assert_parity(got, ref, 1e-5, time_axis=1, what=kind)
+
+
+@pytest.mark.parametrize("kind", SPECIAL)
+def test_special_cases_decode(kind):
+    kla = _kla()
+    x = _special_inputs(kind, T=60)
+    d = {k: torch.from_numpy(v).to(DEV) for k, v in x.items()}
+    lam, eta = d["lam0"].clone(), d["eta0"].clone()
+    mu, var = torch.empty_like(lam), torch.empty_like(lam)
+    mus = []
+    for t in range(x["a"].shape[1]):
+        kla.scan_step(*(d[k][:, t].contiguous() for k in wl.INPUT_NAMES), lam, eta, mu_out=mu, var_out=var)
+        mus.append(mu.clone())
+    torch.cuda.synchronize()
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    got = {"mu": torch.stack(mus, 1).double().cpu().numpy()}
+    parity.assert_parity(got, {"mu": ref["mu"]}, 1e-5, time_axis=1, what=kind)
+    assert np.max(np.abs(lam.double().cpu().numpy() - ref["lam"][:, -1]) / ref["lam"][:, -1]) <= 1e-5

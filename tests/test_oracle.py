@@ -54,3 +54,25 @@ def test_empty_and_bad_shapes(orc):
     assert out["lam"].shape == (1, 0, 1, 4)
     with pytest.raises(ValueError):
         orc.forward(np.zeros((1, 2, 1, 4)), z, z, z, 1.0, 0.0)
+
+
+def test_moebius_factorization():
+    """M_t = [[1, phi], [0, 1]] [[1, 0], [p, a^2]] (update after predict) and
+    the information row of the 3x3 token matrix is b times the predicted
+    denominator row plus a times the old information row -- the forms the
+    CUDA kernels append tokens with -- in exact rational arithmetic."""
+    from fractions import Fraction as F
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        a, b = (F(int(rng.integers(-9, 10)), int(rng.integers(1, 8))) for _ in range(2))
+        p, phi = (F(int(rng.integers(0, 10)), int(rng.integers(1, 8))) for _ in range(2))
+        M = [[1 + p * phi, a * a * phi], [p, a * a]]
+        U = [[1, phi], [0, 1]]
+        P = [[1, 0], [p, a * a]]
+        UP = [[sum(U[i][k] * P[k][j] for k in range(2)) for j in range(2)] for i in range(2)]
+        assert UP == M
+        m = [[F(int(rng.integers(-5, 6)), int(rng.integers(1, 5))) for _ in range(2)] for _ in range(2)]
+        g = [F(int(rng.integers(-5, 6)), int(rng.integers(1, 5))) for _ in range(2)]
+        d = [p * m[0][j] + a * a * m[1][j] for j in range(2)]
+        direct = [b * p * m[0][j] + b * a * a * m[1][j] + a * g[j] for j in range(2)]
+        assert direct == [b * d[j] + a * g[j] for j in range(2)]
