@@ -361,7 +361,7 @@ def run_ours(args):
         e2e = {"value": tc_all / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_s * 1e3,
                "how": "scan_forward on pinned host tensors (C ABI kla_scan_forward_host): the sequence in "
-                      "8 blocks, H2D of a, p, phi, b (+ lam0, eta0), scan, D2H of lambda, eta, mu, var "
+                      "16 blocks, H2D of a, p, phi, b (+ lam0, eta0), scan, D2H of lambda, eta, mu, var "
                       "pipelined on three streams, then a stream sync; wall clock"}
     decode = None
     if not args.no_decode:

@@ -249,7 +249,7 @@ cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &m
     auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, W, NS, kSG>;
     cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    const int64_t grid = std::min<int64_t>(prm.ntiles, sm_count());
+    const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
     kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
     return cudaGetLastError();
 }
@@ -266,6 +266,48 @@ bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt,
     return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Runs per tile for the streaming kernel: the number P <= KLA_STREAM_MAX_PARTS
+// of runs per tile whose units (tiles x P) fill the SMs' rounds best, among
+// those that keep at least 8 chunks per run; 1 when there are fewer than two
+// tiles per SM (a later run's predecessor must have been ticketed a full
+// round earlier, or the run would wait).  Ties go to fewer runs.
+#ifndef KLA_STREAM_MAX_PARTS
+#define KLA_STREAM_MAX_PARTS 4
+#endif
+int stream_parts(int64_t ntiles, int64_t nchunks) {
+    const int64_t G = sm_count();
+    if (ntiles < 2 * G) return 1;
+    int best = 1;
+    double best_balance = 0.0;
+    for (int P = 1; P <= KLA_STREAM_MAX_PARTS; ++P) {
+        if (P > 1 && (nchunks + P - 1) / P < 8) break;
+        const int64_t U = ntiles * P;
+        const int64_t rounds = (U + G - 1) / G;
+        const double balance = (double)U / (double)(rounds * G);
+        if (balance > best_balance + 0.01) {
+            best = P;
+            best_balance = balance;
+        }
+    }
+    return best;
+}
+
+// Workspace of the streaming kernel when it splits tiles into runs: a header
+// (ticket), one ready flag per (tile, run boundary), the states at the run
+// boundaries.
+struct StreamWs {
+    size_t flags_off = 0, state_off = 0, clear_bytes = 0, total = 0;
+};
+StreamWs stream_ws_layout(int64_t ntiles, int parts) {
+    StreamWs w;
+    const size_t nb = (size_t)ntiles * (size_t)(parts - 1);
+    w.flags_off = kHeaderBytes;
+    w.state_off = w.flags_off + round_up(nb * sizeof(unsigned), 256);
+    w.clear_bytes = w.state_off;
+    w.total = w.state_off + round_up(nb * 64 * sizeof(float), 256);
+    return w;
 }
 
 // 2: the channel-owning streaming kernel -- its TMA geometry holds (16-byte
@@ -328,7 +370,9 @@ KLA_API kla_status_t kla_scan_forward_workspace_size(int64_t B, int64_t T, int64
     }
     FwdLayout lay;
     if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
-    *bytes = lay.total;
+    const int64_t ntiles32 = B * ((HN + 31) / 32);
+    const StreamWs sw = stream_ws_layout(ntiles32, 4);  // the most runs the streaming kernel uses
+    *bytes = std::max(lay.total, sw.total);
     return KLA_OK;
 }
 
@@ -358,7 +402,9 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
 
     FwdLayout lay;
     if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
-    if (!workspace || workspace_bytes < lay.total) return KLA_ERR_WORKSPACE_TOO_SMALL;
+    size_t need = 0;
+    if (kla_scan_forward_workspace_size(B, T, H, N, in_dtype, &need) != KLA_OK) return KLA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need) return KLA_ERR_WORKSPACE_TOO_SMALL;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KLA_ERR_MISALIGNED;
     if (T > INT32_MAX || HN > INT32_MAX || B > INT32_MAX || lay.nct > INT32_MAX ||
         lay.nchunks > INT32_MAX)
@@ -404,6 +450,18 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
             sp.nct = (int)((HN + 31) / 32);
             sp.nchunks = (int)((T + kSL - 1) / kSL);
             sp.wait_ns = g_wait_ns.load();
+            sp.parts = stream_parts(sp.ntiles, sp.nchunks);
+            sp.chunks_per_part = (sp.nchunks + sp.parts - 1) / sp.parts;
+            sp.nunits = sp.ntiles * sp.parts;
+            sp.ticket = reinterpret_cast<unsigned *>(ws);
+            sp.part_flags = nullptr;
+            sp.part_state = nullptr;
+            if (sp.parts > 1) {
+                const StreamWs sw = stream_ws_layout(sp.ntiles, sp.parts);
+                sp.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
+                sp.part_state = reinterpret_cast<float *>(ws + sw.state_off);
+                if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
+            }
             const cudaError_t es = in_dtype == KLA_F32 ? launch_forward_stream<float>(sp, smaps, st)
                                                        : launch_forward_stream<__nv_bfloat16>(sp, smaps, st);
             return es == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
@@ -521,7 +579,9 @@ KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int6
     // outputs come from the caching allocator (aligned); only the inputs are passed here
     *kernel = forward_kernel_choice(B, T, HN, dtype_size(in_dtype), a, p, phi, b, nullptr, nullptr, nullptr,
                                     nullptr);
-    *launches = *kernel == 2 ? 1 : 2;
+    *launches = 2;  // chunked kernel: workspace clear + scan
+    if (*kernel == 2)
+        *launches = stream_parts(B * ((HN + 31) / 32), (T + kSL - 1) / kSL) > 1 ? 2 : 1;
     return KLA_OK;
 }
 

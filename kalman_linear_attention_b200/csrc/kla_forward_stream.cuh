@@ -26,12 +26,16 @@
 //                   also clip ragged edges), so the chunk warps do no global
 //                   address arithmetic.
 //
-// No global flags, fences or look-back: the W warps overlap their passes
-// while the producer keeps HBM busy.  Chunk aggregates are formed and applied
-// exactly as in kla_forward_kernel (one thread's run = the whole chunk here).
-// A CTA with more than one tile processes them one after another.  Every
-// mbarrier wait is bounded by the wait limit (a timeout records
-// KLA_ERR_TIMEOUT and the CTA carries on, so nothing can hang).
+// Within a tile no global flags, fences or look-back: the W warps overlap
+// their passes while the producer keeps HBM busy.  Chunk aggregates are formed
+// and applied exactly as in kla_forward_kernel (one thread's run = the whole
+// chunk here).  A CTA with more than one work unit processes them one after
+// another.  When tiles do not divide evenly over the SMs, each tile's
+// sequence is cut into a few runs taken by ticket, run-major, so that a run
+// after the first finds the state published by the previous run (one bounded
+// global wait per run; deadlock-free because a run only waits on a run with a
+// smaller ticket).  Every wait is bounded by the wait limit (a timeout
+// records KLA_ERR_TIMEOUT and the CTA carries on, so nothing can hang).
 #pragma once
 
 #include "kla_forward.cuh"
@@ -61,6 +65,16 @@ struct StreamParams {
     int nchunks;                   // ceil(T / L)
     int write_mu, write_var;       // outputs 2 / 3 requested
     uint64_t wait_ns;
+    // Work units.  parts == 1: unit = tile, CTA c takes tiles c, c + grid, ...
+    // parts > 1: each tile's chunks are cut into `parts` consecutive runs of
+    // chunks_per_part; unit u = part * ntiles + tile is taken by ticket (part
+    // major), and a run after the first enters with the state the previous run
+    // of the same tile published in part_state (flag part_flags).
+    int parts, chunks_per_part;
+    int64_t nunits;                // ntiles * parts
+    unsigned *ticket;              // parts > 1: unit counter (zeroed per call)
+    unsigned *part_flags;          // [ntiles][parts - 1], zeroed per call
+    float *part_state;             // [ntiles][parts - 1][2][32]
 };
 
 template <typename Tin, int L, int W, int NS, int G>
@@ -79,7 +93,8 @@ struct StreamTile {
     static constexpr int OUTBUF_BYTES = 4 * OUTBOX_BYTES;           // four outputs
     static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][32] fp32
     static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][32] fp32
-    static constexpr int BAR_OFF = align_up(CARRY_OFF + W * 2 * CW * 4, 128);  // full, empty, carry
+    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: unit (int64), chunk (int64)
+    static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128); // full, empty, carry
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
 
@@ -100,14 +115,12 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     uint64_t *empty = full + NS;
     uint64_t *carry_bar = empty + NS;
     float *slots = reinterpret_cast<float *>(smem + Cfg::CARRY_OFF);
+    int64_t *meta_unit = reinterpret_cast<int64_t *>(smem + Cfg::META_OFF);  // -1: no more work
+    int64_t *meta_chunk = meta_unit + NS;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
-    const int64_t my_tiles = prm.ntiles > blockIdx.x
-                                 ? (prm.ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int64_t my_chunks = my_tiles * prm.nchunks;
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -122,19 +135,49 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane != 0) return;
-#pragma unroll 1
-        for (int64_t j = 0; j < my_chunks; ++j) {
-            const int s = (int)(j % NS);
-            if (j >= NS) mbar_wait_or_flag(&empty[s], (unsigned)((j / NS - 1) & 1), prm.wait_ns);
-            const int64_t tile = blockIdx.x + (j / prm.nchunks) * gridDim.x;
-            const int64_t chunk = j % prm.nchunks;
+        int64_t seq = 0;  // chunks (and end markers) handed to the chunk warps
+        auto claim = [&]() -> int {
+            const int s = (int)(seq % NS);
+            if (seq >= NS) mbar_wait_or_flag(&empty[s], (unsigned)((seq / NS - 1) & 1), prm.wait_ns);
+            ++seq;
+            return s;
+        };
+        auto load = [&](int64_t unit, int64_t chunk) {
+            const int s = claim();
+            const int64_t tile = unit % prm.ntiles;
             const int bb = (int)(tile / prm.nct);
             const int ct = (int)(tile - (int64_t)bb * prm.nct);
+            meta_unit[s] = unit;
+            meta_chunk[s] = chunk;
             Tin *stage = reinterpret_cast<Tin *>(smem + s * Cfg::STAGE_BYTES);
             mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, (int)(chunk * L), bb, &full[s]);
+        };
+        if (prm.parts == 1) {
+#pragma unroll 1
+            for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x)
+#pragma unroll 1
+                for (int64_t c = 0; c < prm.nchunks; ++c) load(u, c);
+        } else {
+#pragma unroll 1
+            for (;;) {
+                const int64_t u = (int64_t)atomicAdd(prm.ticket, 1u);
+                if (u >= prm.nunits) break;
+                const int64_t c0 = (u / prm.ntiles) * prm.chunks_per_part;
+                const int64_t c1 = c0 + prm.chunks_per_part < prm.nchunks ? c0 + prm.chunks_per_part
+                                                                          : (int64_t)prm.nchunks;
+#pragma unroll 1
+                for (int64_t c = c0; c < c1; ++c) load(u, c);
+            }
+        }
+        // one end marker for each chunk warp
+#pragma unroll 1
+        for (int k = 0; k < W; ++k) {
+            const int s = claim();
+            meta_unit[s] = -1;
+            mbar_arrive(&full[s]);
         }
         return;
     }
@@ -144,11 +187,14 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
     int group_seq = 0;  // output groups this warp has committed (bulk groups are per thread: lane 0)
 #pragma unroll 1
-    for (int64_t j = w; j < my_chunks; j += W) {
+    for (int64_t j = w;; j += W) {
         const int s = (int)(j % NS);
         mbar_wait_or_flag(&full[s], (unsigned)((j / NS) & 1), prm.wait_ns);
-        const int64_t tile = blockIdx.x + (j / prm.nchunks) * gridDim.x;
-        const int64_t chunk = j % prm.nchunks;
+        const int64_t unit = meta_unit[s];
+        if (unit < 0) break;
+        const int64_t chunk = meta_chunk[s];
+        const int64_t tile = unit % prm.ntiles;
+        const int64_t part = unit / prm.ntiles;
         const int64_t bb = tile / prm.nct;
         const int64_t ct = tile - bb * prm.nct;
         const int64_t t0 = chunk * L;
@@ -156,9 +202,14 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
         const int64_t ch = ct * 32 + lane;
         const bool cvalid = ch < prm.HN;
         const Tin *stage = reinterpret_cast<const Tin *>(smem + s * Cfg::STAGE_BYTES);
+        const int64_t first = part * prm.chunks_per_part;  // first chunk of this unit
+        const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
+                                                                         : (int64_t)prm.nchunks) - 1;
 
-        // State entering chunk j (from the previous chunk's warp, or the prior
-        // at a tile's first chunk); hands the state leaving it to the next warp.
+        // State entering chunk j -- from the previous chunk's warp, from the
+        // prior at a tile's first chunk, or from the previous run of the tile
+        // at a later run's first chunk -- and the state leaving it, handed to
+        // the next warp (and published for the next run at a run's end).
         auto chunk_carry = [&](const Agg &g, float &lam, float &eta) {
             if (j > 0) {
                 const int ps = (int)((j - 1) % W);
@@ -169,6 +220,16 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             if (chunk == 0) {
                 lam = cvalid ? prm.lam0[bb * prm.HN + ch] : 1.f;
                 eta = cvalid ? prm.eta0[bb * prm.HN + ch] : 0.f;
+            } else if (chunk == first) {
+                const int64_t slot = tile * (prm.parts - 1) + (part - 1);
+                if (warp_wait_flags(lane == 0 ? prm.part_flags + slot : nullptr, prm.wait_ns)) {
+                    lam = __ldcg(prm.part_state + slot * 64 + lane);
+                    eta = __ldcg(prm.part_state + slot * 64 + 32 + lane);
+                } else {
+                    lam = __int_as_float(0x7fc00000);
+                    eta = lam;
+                    if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
+                }
             }
             float lo = lam, eo = eta;
             agg_apply(g, lo, eo);
@@ -177,6 +238,14 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             slots[ms * 64 + 32 + lane] = eo;
             __syncwarp();
             if (lane == 0) mbar_arrive(&carry_bar[ms]);
+            if (chunk == last && part + 1 < prm.parts) {
+                const int64_t slot = tile * (prm.parts - 1) + part;
+                prm.part_state[slot * 64 + lane] = lo;
+                prm.part_state[slot * 64 + 32 + lane] = eo;
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(prm.part_flags + slot, 1u);
+            }
         };
 
         // Output group q of this chunk (tokens q*G .. q*G+G-1): claim a free

@@ -64,8 +64,10 @@ DeviceQueues *device_queues() {
 
 int64_t pick_block(int64_t T, int64_t t_block) {
     if (t_block > 0) return t_block < T ? t_block : T;
-    // about eight blocks, whole chunks of 64 tokens, at least 64 tokens
-    int64_t tb = (T + 7) / 8;
+    // about sixteen blocks (the first copy in and the last copy out are not
+    // overlapped: ~1/16 of the transfer each), whole chunks of 64 tokens, at
+    // least 64 tokens
+    int64_t tb = (T + 15) / 16;
     tb = (tb + 63) / 64 * 64;
     if (tb < 64) tb = 64;
     return tb < T ? tb : T;

@@ -296,3 +296,26 @@ def test_special_cases_decode(kind):
     got = {"mu": torch.stack(mus, 1).double().cpu().numpy()}
     parity.assert_parity(got, {"mu": ref["mu"]}, 1e-5, time_axis=1, what=kind)
     assert np.max(np.abs(lam.double().cpu().numpy() - ref["lam"][:, -1]) / ref["lam"][:, -1]) <= 1e-5
+
+
+def test_run_split_parity():
+    """320 tiles of 32 channels do not divide evenly over the SMs, so the
+    streaming kernel cuts each tile's sequence into runs taken by ticket; a
+    run enters with the state the previous run published.  Every element
+    against the oracle, and the plan reports the extra clear launch."""
+    kla = _kla()
+    w = wl.WORKLOADS["tiny"].with_shape(B=10, T=1024, H=1, N=1024)
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(v).to(DEV) for k, v in x.items()}
+    kernel, launches = kla.forward_plan(d["a"], d["p"], d["phi"], d["b"])
+    assert kernel == 2
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out)}
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], threads=8)
+    parity.assert_parity(got, ref, 1e-5, time_axis=1, what="run split")
+    print("plan", kernel, launches)
+    again = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    for a_, b_ in zip(out, again):
+        assert torch.equal(a_, b_)  # deterministic despite dynamic tickets
