@@ -68,8 +68,13 @@ static_assert(kCkpt >= 1 && kCkpt <= 32, "checkpoint interval must be 1..32");
 #ifndef KLA_STREAM_W_BF16
 #define KLA_STREAM_W_BF16 11
 #endif
-#ifndef KLA_STREAM_G
-#define KLA_STREAM_G 4
+// Tokens per output box (one TMA store per output per box): 8 for fp32
+// (measured 4-6% faster than 4 on the long workload, same-box A/B).
+#ifndef KLA_STREAM_G_F32
+#define KLA_STREAM_G_F32 8
+#endif
+#ifndef KLA_STREAM_G_BF16
+#define KLA_STREAM_G_BF16 4
 #endif
 #ifndef KLA_STREAM_SMEM
 #define KLA_STREAM_SMEM (227 * 1024)
@@ -78,16 +83,19 @@ static_assert(kCkpt >= 1 && kCkpt <= 32, "checkpoint interval must be 1..32");
 #define KLA_STREAM_MAX_STAGES 24
 #endif
 constexpr int kSL = KLA_STREAM_L;
-constexpr int kSG = KLA_STREAM_G;
 template <typename Tin> constexpr int stream_warps() {
     return sizeof(Tin) == 4 ? KLA_STREAM_W_F32 : KLA_STREAM_W_BF16;
+}
+template <typename Tin> constexpr int stream_group() {
+    return sizeof(Tin) == 4 ? KLA_STREAM_G_F32 : KLA_STREAM_G_BF16;
 }
 // Ring stages that fit beside the per-warp output buffers and carry slots.
 template <typename Tin>
 constexpr int stream_stages() {
     constexpr int W = stream_warps<Tin>();
+    constexpr int G = stream_group<Tin>();
     const int stage = 4 * kSL * 32 * (int)sizeof(Tin);
-    const int fixed = W * 2 * 4 * kSG * 32 * 4 + W * 2 * 32 * 4 + W * 8 + 2048;
+    const int fixed = W * 2 * 4 * G * 32 * 4 + W * 2 * 32 * 4 + W * 8 + 2048;
     const int ns = (KLA_STREAM_SMEM - fixed) / stage;
     return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
 }
@@ -243,10 +251,11 @@ int sm_count() {
 template <typename Tin>
 cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &maps, cudaStream_t stream) {
     constexpr int W = stream_warps<Tin>();
+    constexpr int G = stream_group<Tin>();
     constexpr int NS = stream_stages<Tin>();
-    using Cfg = kla::StreamTile<Tin, kSL, W, NS, kSG>;
+    using Cfg = kla::StreamTile<Tin, kSL, W, NS, G>;
     static_assert(NS >= 2 && Cfg::SMEM <= 227 * 1024, "stream kernel shared memory");
-    auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, W, NS, kSG>;
+    auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, W, NS, G>;
     cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
@@ -441,7 +450,9 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
         for (int k = 0; k < 4 && ok; ++k) ok = encode_stream_map(&smaps.in[k], ins4[k], tdt, esz, B, T, HN, kSL);
         float *outs4[4] = {lambda_out, eta_out, mu_out, var_out};
         for (int k = 0; k < 4 && ok; ++k)
-            if (outs4[k]) ok = encode_stream_map(&smaps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN, kSG);
+            if (outs4[k])
+                ok = encode_stream_map(&smaps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN,
+                                       in_dtype == KLA_F32 ? stream_group<float>() : stream_group<__nv_bfloat16>());
         if (ok) {
             kla::StreamParams sp;
             sp.lam0 = lambda0; sp.eta0 = eta0;
