@@ -540,15 +540,27 @@ KLA_API kla_status_t kla_scan_step(const void *a, const void *p, const void *phi
     const int threads = 256;
     const int64_t work = vec ? C / 4 : C;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((work + threads - 1) / threads, 148 * 16));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (in_dtype == KLA_F32) {
-        if (vec) kla::kla_step_vec4_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(prm);
-        else kla::kla_step_scalar_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(prm);
-    } else {
-        if (vec) kla::kla_step_vec4_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(prm);
-        else kla::kla_step_scalar_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(prm);
-    }
-    return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+    // Programmatic dependent launch: consecutive decode steps overlap the next
+    // step's launch and input prefetch with the current step's tail (the
+    // kernels wait for the preceding grid before touching the state).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (in_dtype == KLA_F32)
+        e = vec ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec4_kernel<float>, prm)
+                : cudaLaunchKernelEx(&cfg, kla::kla_step_scalar_kernel<float>, prm);
+    else
+        e = vec ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec4_kernel<__nv_bfloat16>, prm)
+                : cudaLaunchKernelEx(&cfg, kla::kla_step_scalar_kernel<__nv_bfloat16>, prm);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
 KLA_API kla_status_t kla_get_error(void *stream) {

@@ -35,11 +35,36 @@ template <> struct Vec4In<__nv_bfloat16> {
     }
 };
 
+// Programmatic dependent launch: the kernel may start while the previous
+// kernel on the stream is still running.  Before `griddepcontrol.wait` it only
+// prefetches its token inputs into L2 (L2 is the point of coherence, so a
+// prefetch can never expose a stale value); every load and store happens
+// after the wait, which guarantees that the previous kernel has completed and
+// its writes are visible.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Four channels per thread; every pointer 16-byte aligned (8 for bf16
 // inputs) and C a multiple of 4.
 template <typename Tin>
 __global__ void __launch_bounds__(256) kla_step_vec4_kernel(const StepParams prm) {
     const int64_t n4 = prm.C >> 2;
+    constexpr int VEC_BYTES = 4 * (int)sizeof(Tin);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x)
+        if ((threadIdx.x & 7) == 0)  // one prefetch per 128-byte line (8 threads x 16 bytes, fp32)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                prefetch_l2(static_cast<const char *>(prm.in[k]) + i * VEC_BYTES);
+    grid_dependency_wait();
+    allow_dependent_launch();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float4 a = Vec4In<Tin>::load(prm.in[0], i);
@@ -64,6 +89,8 @@ __global__ void __launch_bounds__(256) kla_step_vec4_kernel(const StepParams prm
 // Any size and alignment: one channel per thread.
 template <typename Tin>
 __global__ void __launch_bounds__(256) kla_step_scalar_kernel(const StepParams prm) {
+    grid_dependency_wait();
+    allow_dependent_launch();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < prm.C;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float a = to_f32(static_cast<const Tin *>(prm.in[0])[i]);
