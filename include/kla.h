@@ -273,13 +273,15 @@ int kla_forward_chunk_tokens(void);
 
 /*
  * Test hook for the forward scan's failure path: in kla_scan_forward calls
- * enqueued afterwards, the chunks with index `chunk` (tokens
- * [chunk * kla_forward_chunk_tokens(), ...)) wait for their carry on a device
- * flag that nothing sets, instead of on the preceding chunk.  The wait runs
- * out after the wait limit, records KLA_ERR_TIMEOUT and writes NaN for that
- * chunk.  Earlier chunks are unaffected; a later chunk is either exact (its
- * look-back composed the stalled chunk's published aggregate) or NaN (it read
- * the stalled chunk's poisoned carry).  -1 (the default) turns the hook off.
+ * enqueued afterwards, the carry into the chunk that starts at token
+ * chunk * kla_forward_chunk_tokens() first waits on a device flag that
+ * nothing sets.  The wait runs out after the wait limit, records
+ * KLA_ERR_TIMEOUT and poisons that chunk's entering state: its outputs are
+ * NaN and earlier tokens are unaffected.  In the chunked kernel a later chunk
+ * is either exact (its look-back composed the stalled chunk's aggregate) or
+ * NaN; in the streaming kernel every later token of the same channels is NaN
+ * (the state is handed from chunk to chunk).  -1 (the default) turns the hook
+ * off.
  */
 kla_status_t kla_debug_stall_chunk(int64_t chunk);
 

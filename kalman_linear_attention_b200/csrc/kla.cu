@@ -461,6 +461,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
             sp.nct = (int)((HN + 31) / 32);
             sp.nchunks = (int)((T + kSL - 1) / kSL);
             sp.wait_ns = g_wait_ns.load();
+            sp.stall_chunk = g_stall_chunk.load() >= 0 ? g_stall_chunk.load() * kL / kSL : -1;
             sp.parts = stream_parts(sp.ntiles, sp.nchunks);
             sp.chunks_per_part = (sp.nchunks + sp.parts - 1) / sp.parts;
             sp.nunits = sp.ntiles * sp.parts;

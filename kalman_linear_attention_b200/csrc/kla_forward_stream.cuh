@@ -75,6 +75,7 @@ struct StreamParams {
     unsigned *ticket;              // parts > 1: unit counter (zeroed per call)
     unsigned *part_flags;          // [ntiles][parts - 1], zeroed per call
     float *part_state;             // [ntiles][parts - 1][2][32]
+    int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
 };
 
 template <typename Tin, int L, int W, int NS, int G>
@@ -217,7 +218,12 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
                 lam = slots[ps * 64 + lane];
                 eta = slots[ps * 64 + 32 + lane];
             }
-            if (chunk == 0) {
+            if (chunk == prm.stall_chunk &&
+                !warp_wait_flags(lane == 0 ? &g_never_set_word : nullptr, prm.wait_ns)) {
+                lam = __int_as_float(0x7fc00000);  // ran out of time: poison what follows
+                eta = lam;
+                if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
+            } else if (chunk == 0) {
                 lam = cvalid ? prm.lam0[bb * prm.HN + ch] : 1.f;
                 eta = cvalid ? prm.eta0[bb * prm.HN + ch] : 0.f;
             } else if (chunk == first) {

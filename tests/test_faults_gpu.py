@@ -61,3 +61,27 @@ def test_stalled_chunk_poisons_only_what_depends_on_it(kla):
     assert kla.get_error() == 0
     got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out2)}
     parity.assert_parity(got, ref, 1e-5, time_axis=1)
+
+
+def test_stalled_chunk_in_streaming_kernel(kla):
+    """The streaming kernel hands the state from chunk to chunk inside the CTA:
+    a carry wait that runs out poisons that chunk and every later token of its
+    channels, leaves earlier tokens exact, and the context stays usable."""
+    kla.debug_force_forward_kernel(2)
+    L = kla.chunk_tokens()
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=512, H=2, N=64)
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
+    kla.debug_stall_chunk(3)
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    assert kla.get_error() == 5
+    kla.debug_stall_chunk(-1)
+    cut = 3 * L
+    ref = oracle.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    ok = {k: o.double().cpu().numpy()[:, :cut] for k, o in zip(parity.OUTPUTS, out)}
+    parity.assert_parity(ok, {k: ref[k][:, :cut] for k in parity.OUTPUTS}, 1e-5, time_axis=1)
+    assert np.isnan(out[0].double().cpu().numpy()[:, cut:]).all()
+    out2 = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out2)}
+    parity.assert_parity(got, ref, 1e-5, time_axis=1)
