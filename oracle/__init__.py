@@ -13,7 +13,11 @@ upcast for fp32 and bf16 inputs).
 Pins: every function here is pinned by ``tests/test_oracle.py`` against exact
 rational arithmetic, closed forms (Riccati fixed point, precision sums, the
 no-process-noise affine case, the no-observation covariance recursion) and
-invariants; none is "parity unpinned".
+invariants.  The gradients (``backward``, reverse mode through the covariance
+form) are pinned against exact forward-mode derivatives (dual numbers over
+Fractions) of the exact Moebius/affine filter, torch autograd through the
+information form, central finite differences of the pinned forward pass, and
+closed-form sums of the a = 1 / p = 0 cases.  None is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -67,6 +71,8 @@ class Oracle:
         lib.kla_oracle_forward.argtypes = [_D] * 10 + [_I64] * 4 + [ctypes.c_int]
         lib.kla_oracle_step.restype = ctypes.c_int
         lib.kla_oracle_step.argtypes = [_D] * 8 + [_I64]
+        lib.kla_oracle_backward.restype = ctypes.c_int
+        lib.kla_oracle_backward.argtypes = [_D] * 16 + [_I64] * 4 + [ctypes.c_int]
         lib.kla_oracle_max_threads.restype = ctypes.c_int
         lib.kla_oracle_max_threads.argtypes = []
         return cls(lib)
@@ -115,6 +121,42 @@ class Oracle:
             raise ValueError(f"kla_oracle_step failed ({rc})")
         return {"lam": lam, "eta": eta, "mu": mu, "var": var}
 
+    def backward(self, a, p, phi, b, lam0, eta0, g_lam=None, g_eta=None, g_mu=None, g_var=None,
+                 threads: int = 1):
+        """Gradients of a loss through the whole-sequence filter.
+
+        ``g_lam``, ``g_eta``, ``g_mu``, ``g_var`` are the loss gradients with
+        respect to the four [B, T, H, N] outputs (None: zero).  Returns a dict
+        with fp64 ``a``, ``p``, ``phi``, ``b`` ([B, T, H, N]) and ``lam0``,
+        ``eta0`` ([B, H, N]): the gradients with respect to each input.
+        """
+        a, p, phi, b = (_f64(x) for x in (a, p, phi, b))
+        if a.ndim != 4 or not (a.shape == p.shape == phi.shape == b.shape):
+            raise ValueError("a, p, phi, b must share one [B, T, H, N] shape")
+        B, T, H, N = a.shape
+        lam0 = _f64(np.broadcast_to(np.asarray(lam0, dtype=np.float64), (B, H, N)))
+        eta0 = _f64(np.broadcast_to(np.asarray(eta0, dtype=np.float64), (B, H, N)))
+        grads = []
+        for g in (g_lam, g_eta, g_mu, g_var):
+            if g is None:
+                grads.append(None)
+                continue
+            g = _f64(g)
+            if g.shape != a.shape:
+                raise ValueError("output gradients must be [B, T, H, N]")
+            grads.append(g)
+        out = {k: np.empty((B, T, H, N), dtype=np.float64) for k in ("a", "p", "phi", "b")}
+        out["lam0"] = np.empty((B, H, N), dtype=np.float64)
+        out["eta0"] = np.empty((B, H, N), dtype=np.float64)
+        gp = [None if g is None else _ptr(g) for g in grads]
+        rc = self.lib.kla_oracle_backward(
+            _ptr(a), _ptr(p), _ptr(phi), _ptr(b), _ptr(lam0), _ptr(eta0), *gp,
+            _ptr(out["a"]), _ptr(out["p"]), _ptr(out["phi"]), _ptr(out["b"]),
+            _ptr(out["lam0"]), _ptr(out["eta0"]), B, T, H, N, int(threads))
+        if rc != 0:
+            raise ValueError(f"kla_oracle_backward failed ({rc})")
+        return out
+
 
 _DEFAULT: Oracle | None = None
 
@@ -133,3 +175,8 @@ def forward(a, p, phi, b, lam0, eta0, threads: int = 1):
 
 def step(a, p, phi, b, lam_state, eta_state):
     return default().step(a, p, phi, b, lam_state, eta_state)
+
+
+def backward(a, p, phi, b, lam0, eta0, g_lam=None, g_eta=None, g_mu=None, g_var=None,
+             threads: int = 1):
+    return default().backward(a, p, phi, b, lam0, eta0, g_lam, g_eta, g_mu, g_var, threads=threads)

@@ -37,6 +37,7 @@
  */
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -127,6 +128,133 @@ int kla_oracle_step(const double *a, const double *p, const double *phi,
         var[ch] = 1.0 / lam_t;
     }
     return 0;
+}
+
+/*
+ * Gradients (reverse mode) of the whole-sequence filter above.
+ *
+ * Given the gradients of a scalar loss with respect to every output
+ * (g_lambda, g_eta, g_mu, g_var, each [B, T, H, N]; a NULL array means a zero
+ * gradient), return the gradients with respect to every input: a, p, phi, b
+ * ([B, T, H, N]) and the prior lambda0, eta0 ([B, H, N]).  The KLA review
+ * claims end-to-end training of the layer ("parallel training" of the filter)
+ * without giving the backward pass; this is the chain rule taken through the
+ * covariance-form steps of kf_token / kf_channel, one token at a time in
+ * reverse, nothing else:
+ *
+ *   state entering token t:  P (variance), m (mean)
+ *   P- = a^2 P + p,  m- = a m,  lambda = 1/P- + phi,  eta = m-/P- + b,
+ *   mu = eta/lambda,  var = 1/lambda,  and the state leaving the token is
+ *   P' = 1/lambda, m' = eta/lambda (the same expressions as var and mu).
+ *
+ * Walking back, (gP', gm') is the gradient flowing into the state that leaves
+ * token t from every later token (zero after the last one).  The prior enters
+ * as P = 1/lambda0, m = eta0/lambda0.  The forward pass is recomputed for each
+ * channel (the states entering every token are kept in a scratch array).
+ * Returns 0 on success, -1 on a bad argument, -2 when scratch memory cannot be
+ * allocated.
+ */
+static void kf_channel_backward(const double *a, const double *p, const double *phi,
+                                const double *b, int64_t T, int64_t stride,
+                                double lam0, double eta0,
+                                const double *g_lam, const double *g_eta,
+                                const double *g_mu, const double *g_var,
+                                double *ga, double *gp, double *gphi, double *gb,
+                                double *g_lam0, double *g_eta0,
+                                double *P_in, double *m_in)
+{
+    /* forward: the state entering each token */
+    double P = 1.0 / lam0, m = eta0 / lam0;
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t k = t * stride;
+        P_in[t] = P;
+        m_in[t] = m;
+        double lam_t, eta_t;
+        kf_token(a[k], p[k], phi[k], b[k], P, m, &lam_t, &eta_t);
+        const double P_out = 1.0 / lam_t, m_out = eta_t / lam_t;
+        P = P_out;
+        m = m_out;
+    }
+    /* reverse */
+    double gP_next = 0.0, gm_next = 0.0;
+    for (int64_t t = T - 1; t >= 0; --t) {
+        const int64_t i = t * stride;
+        const double at = a[i], pt = p[i];
+        const double P_prev = P_in[t], m_prev = m_in[t];
+        /* recompute the token */
+        const double P_pred = at * at * P_prev + pt;
+        const double m_pred = at * m_prev;
+        const double lam = 1.0 / P_pred + phi[i];
+        const double eta = m_pred / P_pred + b[i];
+        /* gradients reaching var (= P') and mu (= m') */
+        const double g_v = (g_var ? g_var[i] : 0.0) + gP_next;
+        const double g_m = (g_mu ? g_mu[i] : 0.0) + gm_next;
+        /* mu = eta / lambda, var = 1 / lambda */
+        const double g_l = (g_lam ? g_lam[i] : 0.0)
+                           - g_v / (lam * lam) - g_m * eta / (lam * lam);
+        const double g_e = (g_eta ? g_eta[i] : 0.0) + g_m / lam;
+        /* lambda = 1/P- + phi, eta = m-/P- + b */
+        gphi[i] = g_l;
+        gb[i] = g_e;
+        const double g_Pp = -g_l / (P_pred * P_pred) - g_e * m_pred / (P_pred * P_pred);
+        const double g_mp = g_e / P_pred;
+        /* P- = a^2 P + p, m- = a m */
+        ga[i] = g_Pp * 2.0 * at * P_prev + g_mp * m_prev;
+        gp[i] = g_Pp;
+        gP_next = g_Pp * at * at;
+        gm_next = g_mp * at;
+    }
+    /* P = 1/lambda0, m = eta0/lambda0 */
+    *g_lam0 = -gP_next / (lam0 * lam0) - gm_next * eta0 / (lam0 * lam0);
+    *g_eta0 = gm_next / lam0;
+}
+
+int kla_oracle_backward(const double *a, const double *p, const double *phi,
+                        const double *b, const double *lam0, const double *eta0,
+                        const double *g_lam, const double *g_eta,
+                        const double *g_mu, const double *g_var,
+                        double *ga, double *gp, double *gphi, double *gb,
+                        double *g_lam0, double *g_eta0,
+                        int64_t B, int64_t T, int64_t H, int64_t N, int nthreads)
+{
+    if (B < 0 || T < 0 || H < 0 || N < 0) return -1;
+    const int64_t HN = H * N;
+    const int64_t C = B * HN;
+    if (C == 0) return 0;
+    if (!lam0 || !eta0 || !g_lam0 || !g_eta0) return -1;
+    if (T > 0 && (!a || !p || !phi || !b || !ga || !gp || !gphi || !gb)) return -1;
+    if (nthreads <= 0) nthreads = 1;
+    int failed = 0;
+#ifdef _OPENMP
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *scratch = (double *)malloc(sizeof(double) * (size_t)(2 * (T > 0 ? T : 1)));
+        if (!scratch) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            failed = 1;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t ch = 0; ch < C; ++ch) {
+            if (!scratch) continue;
+            const int64_t bi = ch / HN;
+            const int64_t hn = ch % HN;
+            const int64_t base = (bi * T) * HN + hn;  /* token 0 of the channel */
+            const double prior_lam = lam0[ch], prior_eta = eta0[ch];
+            kf_channel_backward(a + base, p + base, phi + base, b + base, T, HN,
+                                prior_lam, prior_eta,
+                                g_lam ? g_lam + base : NULL, g_eta ? g_eta + base : NULL,
+                                g_mu ? g_mu + base : NULL, g_var ? g_var + base : NULL,
+                                ga + base, gp + base, gphi + base, gb + base,
+                                g_lam0 + ch, g_eta0 + ch, scratch, scratch + (T > 0 ? T : 1));
+        }
+        free(scratch);
+    }
+    return failed ? -2 : 0;
 }
 
 /* Number of threads an OpenMP region may use here (1 without OpenMP). */

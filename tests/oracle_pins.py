@@ -339,6 +339,230 @@ def pin_invariants(orc):
         _scaled_close(out["mu"] * out["lam"], out["eta"], 1e-14, f"{name} mu*lam")
 
 
+# ------------------------------------------------------ gradients (backward)
+class Dual:
+    """Exact forward-mode derivative: value + eps * derivative, eps^2 = 0, with
+    Fraction components (so a derivative of the exact filter is exact too)."""
+
+    __slots__ = ("v", "d")
+
+    def __init__(self, v, d=0):
+        self.v, self.d = Fr(v), Fr(d)
+
+    @staticmethod
+    def _of(x):
+        return x if isinstance(x, Dual) else Dual(x)
+
+    def __add__(self, o):
+        o = Dual._of(o)
+        return Dual(self.v + o.v, self.d + o.d)
+
+    __radd__ = __add__
+
+    def __sub__(self, o):
+        o = Dual._of(o)
+        return Dual(self.v - o.v, self.d - o.d)
+
+    def __rsub__(self, o):
+        return Dual._of(o) - self
+
+    def __mul__(self, o):
+        o = Dual._of(o)
+        return Dual(self.v * o.v, self.d * o.v + self.v * o.d)
+
+    __rmul__ = __mul__
+
+    def __truediv__(self, o):
+        o = Dual._of(o)
+        return Dual(self.v / o.v, (self.d * o.v - self.v * o.d) / (o.v * o.v))
+
+    def __rtruediv__(self, o):
+        return Dual._of(o) / self
+
+
+_GRAD_INPUTS = ("a", "p", "phi", "b")
+
+
+def _exact_loss_gradient(fr, w, bi, h, n):
+    """Exact gradient of L = sum_t w_lam lam_t + w_eta eta_t + w_mu mu_t +
+    w_var var_t for one channel, one forward-mode pass per input element
+    (the exact Moebius/affine filter with a Dual seeded on that element)."""
+    T = fr["a"].shape[1]
+    sl = (bi, slice(None), h, n)
+    base = {k: list(fr[k][sl]) for k in _GRAD_INPUTS}
+    base["lam0"], base["eta0"] = fr["lam0"][bi, h, n], fr["eta0"][bi, h, n]
+    wl_, we, wm, wv = (list(x[sl]) for x in w)
+
+    def loss_derivative(key, t):
+        args = {k: ([Dual(x) for x in v] if isinstance(v, list) else Dual(v)) for k, v in base.items()}
+        if t is None:
+            args[key] = Dual(base[key], 1)
+        else:
+            args[key][t] = Dual(base[key][t], 1)
+        lam, eta = exact_moebius_filter(args["a"], args["p"], args["phi"], args["b"],
+                                        args["lam0"], args["eta0"])
+        tot = Fr(0)
+        for s in range(T):
+            tot += (wl_[s] * lam[s] + we[s] * eta[s] + wm[s] * (eta[s] / lam[s])
+                    + wv[s] * (1 / lam[s])).d
+        return tot
+
+    g = {k: [loss_derivative(k, t) for t in range(T)] for k in _GRAD_INPUTS}
+    g["lam0"] = loss_derivative("lam0", None)
+    g["eta0"] = loss_derivative("eta0", None)
+    return g
+
+
+def pin_backward_exact_dual(orc, seeds=(4, 5)):
+    """Reverse-mode gradients of the oracle == exact forward-mode derivatives
+    (Dual numbers over Fractions) of the exact Moebius/affine filter, for every
+    input element, with random rational output gradients (B=2, per-channel
+    priors and negative a as in the forward pin)."""
+    for seed in seeds:
+        fr = random_rational_problem(seed, B=2, T=5, H=1, N=2)
+        rng = np.random.default_rng(seed + 100)
+        shape = fr["a"].shape
+        w = []
+        for _ in range(4):
+            arr = np.empty(shape, dtype=object)
+            for idx in np.ndindex(shape):
+                arr[idx] = _random_fraction(rng, -5, 5, 4)
+            w.append(arr)
+        B, T, H, N = shape
+        exact = {k: np.empty(shape, dtype=object) for k in _GRAD_INPUTS}
+        exact["lam0"] = np.empty((B, H, N), dtype=object)
+        exact["eta0"] = np.empty((B, H, N), dtype=object)
+        for bi in range(B):
+            for h in range(H):
+                for n in range(N):
+                    g = _exact_loss_gradient(fr, w, bi, h, n)
+                    for k in _GRAD_INPUTS:
+                        exact[k][bi, :, h, n] = g[k]
+                    exact["lam0"][bi, h, n] = g["lam0"]
+                    exact["eta0"][bi, h, n] = g["eta0"]
+        f64 = {k: _to_f64(v) for k, v in fr.items()}
+        got = orc.backward(f64["a"], f64["p"], f64["phi"], f64["b"], f64["lam0"], f64["eta0"],
+                           *[_to_f64(x) for x in w])
+        for k in exact:
+            ref = _to_f64(exact[k])
+            _scaled_close(got[k], ref, 1e-12, f"exact gradient d/d{k} (seed {seed})",
+                          axis=1 if ref.ndim == 4 else None)
+
+
+def _torch_info_form_loss(a, p, phi, b, lam0, eta0, w):
+    """The information form of the filter written with torch fp64 ops (the
+    Moebius precision map and the precision-ratio gate), for autograd."""
+    import torch
+    lam, eta = lam0, eta0
+    tot = torch.zeros((), dtype=torch.float64)
+    for t in range(a.shape[1]):
+        at, pt, ft, bt = a[:, t], p[:, t], phi[:, t], b[:, t]
+        gate = at / (at * at + pt * lam)
+        lam_new = ((1 + pt * ft) * lam + at * at * ft) / (pt * lam + at * at)
+        eta = gate * eta + bt
+        lam = lam_new
+        tot = tot + (w[0][:, t] * lam + w[1][:, t] * eta + w[2][:, t] * (eta / lam)
+                     + w[3][:, t] / lam).sum()
+    return tot
+
+
+def pin_backward_autograd(orc):
+    """Oracle gradients == torch autograd through the information form
+    (Moebius map + gate, fp64) on a random problem with every output gradient
+    present, and again with only some present (the others zero)."""
+    import torch
+    rng = np.random.default_rng(77)
+    B, T, H, N = 2, 40, 2, 3
+    x = {"a": rng.uniform(0.5, 1.0, (B, T, H, N)) * np.where(rng.random((B, T, H, N)) < 0.2, -1, 1),
+         "p": np.exp(rng.uniform(np.log(1e-3), 0, (B, T, H, N))),
+         "phi": np.exp(rng.uniform(np.log(1e-2), np.log(10), (B, T, H, N))),
+         "b": rng.standard_normal((B, T, H, N)),
+         "lam0": np.exp(rng.uniform(-1, 1, (B, H, N))),
+         "eta0": rng.standard_normal((B, H, N))}
+    w_all = [rng.standard_normal((B, T, H, N)) for _ in range(4)]
+    for present in ((0, 1, 2, 3), (2,), (0, 3), (1,)):
+        w = [w_all[i] if i in present else None for i in range(4)]
+        got = orc.backward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], *w)
+        tx = {k: torch.tensor(v, dtype=torch.float64, requires_grad=True) for k, v in x.items()}
+        tw = [torch.tensor(v if v is not None else np.zeros((B, T, H, N)), dtype=torch.float64)
+              for v in w]
+        loss = _torch_info_form_loss(tx["a"], tx["p"], tx["phi"], tx["b"], tx["lam0"], tx["eta0"], tw)
+        loss.backward()
+        for k in x:
+            ref = tx[k].grad.numpy()
+            _scaled_close(got[k], ref, 1e-11, f"autograd d/d{k} (outputs {present})",
+                          axis=1 if ref.ndim == 4 else None)
+
+
+def pin_backward_finite_difference(orc):
+    """Oracle gradients == central finite differences of the oracle's own
+    (pinned) forward pass, on sampled elements of every input, for a loss on
+    all four outputs with workload-like inputs."""
+    rng = np.random.default_rng(91)
+    w = wl.WORKLOADS["lm_layer"].with_shape(B=2, T=48, H=1, N=3)
+    x = dict(wl.generate(w))
+    x = {k: np.asarray(v, dtype=np.float64) for k, v in x.items()}
+    x["lam0"] = np.exp(rng.uniform(-1, 1, x["lam0"].shape))
+    x["eta0"] = rng.standard_normal(x["eta0"].shape)
+    gw = [rng.standard_normal(x["a"].shape) for _ in range(4)]
+    got = orc.backward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], *gw)
+
+    def loss(arrs):
+        o = orc.forward(arrs["a"], arrs["p"], arrs["phi"], arrs["b"], arrs["lam0"], arrs["eta0"])
+        return math.fsum(float((g * o[k]).sum()) for g, k in zip(gw, ("lam", "eta", "mu", "var")))
+
+    for k in ("a", "p", "phi", "b", "lam0", "eta0"):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, s)) for s in x[k].shape)
+            h = 1e-6 * max(abs(x[k][idx]), 1e-3)
+            up = {kk: v.copy() for kk, v in x.items()}
+            dn = {kk: v.copy() for kk, v in x.items()}
+            up[k][idx] += h
+            dn[k][idx] -= h
+            fd = (loss(up) - loss(dn)) / (2 * h)
+            g = got[k][idx]
+            assert abs(g - fd) <= 2e-5 * (abs(fd) + 1e-3), f"d/d{k}{idx}: {g} vs finite difference {fd}"
+
+
+def pin_backward_closed_forms(orc):
+    """Textbook sums: with a = 1, p = 0 the precision and information are
+    running sums, so d/dphi_s = sum_{t>=s} g_lam_t and d/db_s = sum_{t>=s} g_eta_t
+    (and the prior collects the full sums); with p = 0 and a loss on the last
+    token only, d lam_T/d phi_s = prod_{j>s} a_j^-2 and d eta_T/d b_s =
+    prod_{j>s} a_j^-1 (the affine case of the Moebius map)."""
+    rng = np.random.default_rng(13)
+    T = 64
+    phi = np.exp(rng.uniform(np.log(1e-2), np.log(10), T))
+    b = rng.standard_normal(T)
+    gl, ge = rng.standard_normal(T), rng.standard_normal(T)
+    got = orc.backward(_as4(np.ones(T)), _as4(np.zeros(T)), _as4(phi), _as4(b), [[[1.5]]], [[[0.2]]],
+                       g_lam=_as4(gl), g_eta=_as4(ge))
+    suf_l = np.array([math.fsum(gl[s:]) for s in range(T)])
+    suf_e = np.array([math.fsum(ge[s:]) for s in range(T)])
+    _scaled_close(got["phi"][0, :, 0, 0], suf_l, 1e-13, "a=1,p=0: d/dphi = suffix sum of g_lam", axis=None)
+    _scaled_close(got["b"][0, :, 0, 0], suf_e, 1e-13, "a=1,p=0: d/db = suffix sum of g_eta", axis=None)
+    assert abs(got["lam0"][0, 0, 0] - suf_l[0]) <= 1e-12 * (abs(suf_l[0]) + 1)
+    assert abs(got["eta0"][0, 0, 0] - suf_e[0]) <= 1e-12 * (abs(suf_e[0]) + 1)
+    a = rng.uniform(0.8, 1.2, T) * np.where(rng.random(T) < 0.3, -1.0, 1.0)
+    last = np.zeros(T)
+    last[-1] = 1.0
+    got = orc.backward(_as4(a), _as4(np.zeros(T)), _as4(phi), _as4(b), [[[0.7]]], [[[0.3]]],
+                       g_lam=_as4(last))
+    ref = np.array([np.prod(a[s + 1:] ** -2.0) for s in range(T)])
+    _rel_close(got["phi"][0, :, 0, 0], ref, 1e-12, "p=0: d lam_T / d phi_s")
+    _rel_close(got["lam0"][0, 0, 0], np.prod(a ** -2.0), 1e-12, "p=0: d lam_T / d lam_0")
+    got = orc.backward(_as4(a), _as4(np.zeros(T)), _as4(phi), _as4(b), [[[0.7]]], [[[0.3]]],
+                       g_eta=_as4(last))
+    ref = np.array([np.prod(1.0 / a[s + 1:]) for s in range(T)])
+    _rel_close(got["b"][0, :, 0, 0], ref, 1e-12, "p=0: d eta_T / d b_s")
+    _rel_close(got["eta0"][0, 0, 0], np.prod(1.0 / a), 1e-12, "p=0: d eta_T / d eta_0")
+    assert np.max(np.abs(got["phi"])) <= 1e-12 * np.max(np.abs(got["b"])), \
+        "p=0: eta does not depend on the precision path"
+
+
+BACKWARD_PINS = [pin_backward_exact_dual, pin_backward_autograd, pin_backward_finite_difference,
+                 pin_backward_closed_forms]
+
 ALL_PINS = [pin_exact_rational, pin_exact_rational_step, pin_riccati, pin_precision_sum,
             pin_no_process_noise, pin_no_observation, pin_gate_derivative, pin_gate_product,
-            pin_invariants]
+            pin_invariants] + BACKWARD_PINS

@@ -76,3 +76,34 @@ def test_moebius_factorization():
         d = [p * m[0][j] + a * a * m[1][j] for j in range(2)]
         direct = [b * p * m[0][j] + b * a * a * m[1][j] + a * g[j] for j in range(2)]
         assert direct == [b * d[j] + a * g[j] for j in range(2)]
+
+
+def test_backward_threads_and_absent_gradients(orc):
+    """Threads split channels only (bitwise equal), and an absent output
+    gradient is the same as a zero one."""
+    w = wl.WORKLOADS["stiff"].with_shape(B=3, T=30)
+    x = wl.generate(w)
+    rng = np.random.default_rng(2)
+    g = [rng.standard_normal(x["a"].shape) for _ in range(4)]
+    args = (x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])
+    one = orc.backward(*args, *g, threads=1)
+    many = orc.backward(*args, *g, threads=4)
+    for k in one:
+        assert np.array_equal(one[k], many[k]), k
+    absent = orc.backward(*args, g[0], None, g[2], None)
+    zeros = orc.backward(*args, g[0], np.zeros_like(g[1]), g[2], np.zeros_like(g[3]))
+    for k in absent:
+        assert np.array_equal(absent[k], zeros[k]), k
+
+
+def test_backward_empty_and_bad_shapes(orc):
+    """T = 0: no outputs, so the prior's gradients are zero."""
+    z = np.zeros((2, 0, 1, 4))
+    out = orc.backward(z, z, z, z, np.ones((2, 1, 4)), np.zeros((2, 1, 4)), z, z, z, z)
+    assert out["a"].shape == (2, 0, 1, 4)
+    assert np.array_equal(out["lam0"], np.zeros((2, 1, 4)))
+    assert np.array_equal(out["eta0"], np.zeros((2, 1, 4)))
+    with pytest.raises(ValueError):
+        orc.backward(np.zeros((1, 2, 1, 4)), z, z, z, 1.0, 0.0)
+    with pytest.raises(ValueError):
+        orc.backward(*(np.zeros((1, 2, 1, 4)),) * 4, 1.0, 0.0, g_mu=np.zeros((1, 3, 1, 4)))

@@ -33,6 +33,24 @@ MUTANTS = {
     "decode step: state read as variance": ("const double P = 1.0 / lam_state[ch];",
                                             "const double P = lam_state[ch];"),
     "decode step: eta not written": ("        eta_state[ch] = eta_t;", "        (void)eta_t;"),
+    # the reverse-mode gradients
+    "backward: later variance gradient dropped": ("+ gP_next;", ";"),
+    "backward: later mean gradient dropped": ("+ gm_next;", ";"),
+    "backward: var term sign": ("- g_v / (lam * lam) - g_m", "+ g_v / (lam * lam) - g_m"),
+    "backward: mu -> eta uses lambda": ("+ g_m / lam;", "+ g_m * lam;"),
+    "backward: mean path dropped from P-": ("- g_e * m_pred / (P_pred * P_pred);", ";"),
+    "backward: d(a^2)/da = a": ("g_Pp * 2.0 * at * P_prev", "g_Pp * at * P_prev"),
+    "backward: mean term of a dropped": ("+ g_mp * m_prev;", ";"),
+    "backward: variance carried by a": ("gP_next = g_Pp * at * at;", "gP_next = g_Pp * at;"),
+    "backward: mean carried without a": ("gm_next = g_mp * at;", "gm_next = g_mp;"),
+    "backward: prior mean term dropped": ("- gm_next * eta0 / (lam0 * lam0);", ";"),
+    "backward: prior information gradient": ("*g_eta0 = gm_next / lam0;", "*g_eta0 = gm_next;"),
+    "backward: phi and b gradients swapped": ("gphi[i] = g_l;\n        gb[i] = g_e;",
+                                               "gphi[i] = g_e;\n        gb[i] = g_l;"),
+    "backward: wrong batch stride": ("(bi * T) * HN + hn;", "bi * HN + hn;"),
+    "backward: prior variance = lambda_0": ("double P = 1.0 / lam0, m", "double P = lam0, m"),
+    "backward: recomputed state carries the variance only": ("m = m_out;", "m = m_out * 0.0 + m;"),
+    "backward: recomputed mean not divided": ("m_out = eta_t / lam_t;", "m_out = eta_t;"),
 }
 
 
