@@ -6,7 +6,8 @@ cross-chunk carry, emit lambda / eta / mu / var) over the long-sequence
 workload (B=1, H=32, N=128, T=65536, fp32): 268.4 M token-channels per GPU,
 8.59 GB of algorithmic HBM traffic.  The same line also reports the recurrent
 decode step (B=256, H=32, N=128, fp32 resident state; 1024 tokens replayed
-from a CUDA graph).
+from a CUDA graph) and the backward scan (kla_scan_backward) of the same
+workload.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -219,7 +220,60 @@ def time_forward(kla, w, dev, steps: int, warmup: int, dist_mod):
         raise RuntimeError("device-side error in the timed region")
     total_ms = t_start.elapsed_time(t_end)
     per_launch = [a.elapsed_time(b) for a, b in ev]
-    return total_ms, per_launch, plan
+    return total_ms, per_launch, plan, outs
+
+
+def backward_bytes_per_tc(w: wl.Workload) -> int:
+    """Bytes the backward scan must move per token-channel with all four
+    output gradients present: read a, p (input dtype), lambda, eta and the
+    four output gradients (fp32); write the four input gradients (input
+    dtype)."""
+    e = 2 if w.dtype == "bf16" else 4
+    return 2 * e + 2 * 4 + 4 * 4 + 4 * e
+
+
+def time_backward(kla, w, dev, outs, steps: int, warmup: int, peak: float):
+    """kla_scan_backward on the forward's lambda / eta with all four output
+    gradients present (the general case), CUDA events per launch."""
+    import torch
+    B, T, H, N = w.B, w.T, w.H, w.N
+    device = dev["a"].device
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 17)
+    grads = [torch.randn((B, T, H, N), generator=gen, device=device) for _ in range(4)]
+    res = [torch.empty((B, T, H, N), dtype=dev["a"].dtype, device=device) for _ in range(4)]
+    res += [torch.empty((B, H, N), device=device) for _ in range(2)]
+    ws = torch.empty(max(kla.backward_workspace_size(B, T, H, N, dev["a"].dtype), 1), dtype=torch.uint8,
+                     device=device)
+    plan = kla.backward_plan(dev["a"], dev["p"])
+    args = (dev["a"], dev["p"], dev["lam0"], dev["eta0"], outs[0], outs[1], *grads)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        kla.scan_backward(*args, out=res, workspace=ws)
+    torch.cuda.synchronize()
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error during backward warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(stream)
+        kla.scan_backward(*args, out=res, workspace=ws)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error in the timed backward region")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    bpt = backward_bytes_per_tc(w)
+    tc = w.token_channels
+    gbs = bpt * tc / (ms * 1e-3) / 1e9
+    del grads, res
+    return {"workload": f"{w.name}: {w.summary}, all four output gradients present",
+            "ms_per_step": ms, "value": tc / (ms * 1e-3), "unit": UNIT, "steps": steps, "warmup": warmup,
+            "kernel": {1: "kla_backward_seq_kernel (one thread per channel)",
+                       2: "kla_backward_stream_kernel (channel-owning streaming, reverse time)"}[plan[0]],
+            "gpu_launches": plan[1] * steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "algorithmic_bytes_per_launch": bpt * tc, "traffic": None},
+            "data": "forward outputs of the timed forward; output gradients from a seeded torch.randn on the device"}
 
 
 def time_e2e(kla, w, host, steps: int):
@@ -335,8 +389,8 @@ def run_ours(args):
 
     sampler = ClockSampler(local)
     sampler.start()
-    total_ms, per_launch, plan = time_forward(kla, w, dev, args.steps, args.warmup,
-                                              dist if world > 1 else None)
+    total_ms, per_launch, plan, fwd_outs = time_forward(kla, w, dev, args.steps, args.warmup,
+                                                        dist if world > 1 else None)
     kernel_name = {1: "kla_forward_kernel (chunked; + its workspace clear kernel, timed together)",
                    2: "kla_forward_stream_kernel (channel-owning streaming)"}[plan[0]]
     clocks = sampler.stop()
@@ -351,6 +405,11 @@ def run_ours(args):
     peak, peak_src = measured_peaks()
     traffic = recorded_traffic(args.workload if not args.tokens else f"{args.workload}@T={args.tokens}",
                                plan[0])
+
+    backward = None
+    if not args.no_backward:
+        backward = time_backward(kla, w, dev, fwd_outs, args.backward_steps, args.warmup, peak)
+    del fwd_outs
 
     e2e = None
     if host is not None:
@@ -395,6 +454,7 @@ def run_ours(args):
         "clocks": clocks,
         "e2e": e2e,
         "decode": decode,
+        "backward": backward,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line))
@@ -452,6 +512,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-steps", type=int, default=50)
     return ap.parse_args(argv)
 
 

@@ -241,6 +241,85 @@ kla_status_t kla_scan_step(const void *a, const void *p, const void *phi, const 
                            int64_t B, int64_t H, int64_t N, void *stream);
 
 /*
+ * Size in bytes of the device workspace kla_scan_backward needs for a problem
+ * of this shape (the run-boundary carries and flags used when the sequence
+ * of a channel tile is split into runs across SMs), written to *bytes.  0 for
+ * an empty problem.  KLA_ERR_INVALID_ARG for negative sizes or a null `bytes`.
+ */
+kla_status_t kla_scan_backward_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                              kla_dtype_t in_dtype, size_t *bytes);
+
+/*
+ * Gradients of a scalar loss through kla_scan_forward (reverse mode).  The
+ * review claims end-to-end parallel training of the layer but gives no
+ * backward pass; this one differentiates the information-form recursion
+ * above.  With D_t = a_t^2 + p_t lambda_{t-1}, r_t = 1/D_t, f_t = a_t r_t:
+ *
+ *   fold        gl_t = g_lambda_t - v_t (g_mu_t mu_t + g_var_t v_t),
+ *               ge_t = g_eta_t + g_mu_t v_t      (v_t = 1/lambda_t, mu_t = eta_t v_t)
+ *   adjoint     E_t = dL/d eta_t    = ge_t + f_{t+1} E_{t+1},
+ *               L_t = dL/d lambda_t = gl_t + f_{t+1}^2 L_{t+1} + c_{t+1} E_{t+1},
+ *               c_t = -p_t f_t r_t eta_{t-1}      (a reverse-time scan)
+ *   inputs      d/d phi_t = L_t,  d/d b_t = E_t,
+ *               d/d a_t = r_t^2 (-2 a_t lambda_{t-1} L_t + (p_t lambda_{t-1} - a_t^2) eta_{t-1} E_t),
+ *               d/d p_t = -r_t^2 lambda_{t-1} (lambda_{t-1} L_t + a_t eta_{t-1} E_t),
+ *               d/d eta_0 = f_1 E_1,  d/d lambda_0 = f_1^2 L_1 + c_1 E_1.
+ *
+ *   a, p           [B, T, H, N] forward inputs, dtype in_dtype (read only);
+ *                  phi and b are not needed (they enter through lambda, eta)
+ *   lambda0, eta0  [B, H, N] fp32 prior of the forward call (read only)
+ *   lambda_out, eta_out
+ *                  [B, T, H, N] fp32 outputs of that forward call (read only)
+ *   g_lambda, g_eta, g_mu, g_var
+ *                  [B, T, H, N] fp32 gradients of the loss with respect to the
+ *                  four forward outputs; NULL = zero (that array is not read)
+ *   grad_a, grad_p, grad_phi, grad_b
+ *                  [B, T, H, N] gradients with respect to the inputs, written
+ *                  in in_dtype (fp32 arithmetic, rounded once on store); NULL =
+ *                  not wanted
+ *   grad_lambda0, grad_eta0
+ *                  [B, H, N] fp32 gradients with respect to the prior, or NULL
+ *   workspace      device scratch of at least
+ *                  kla_scan_backward_workspace_size(...) bytes, 256-byte
+ *                  aligned (may be NULL when that size is 0); contents on
+ *                  entry do not matter.  Concurrent calls need their own.
+ *
+ * B*H*N == 0 is valid (nothing is enqueued).  T == 0 writes zero prior
+ * gradients.  Outputs must not overlap the inputs, the workspace or each
+ * other (KLA_ERR_INVALID_ARG).  Same preconditions as the forward call; the
+ * forward outputs are trusted as given.
+ */
+kla_status_t kla_scan_backward(const void *a, const void *p, kla_dtype_t in_dtype,
+                               const float *lambda0, const float *eta0,
+                               const float *lambda_out, const float *eta_out,
+                               const float *g_lambda, const float *g_eta,
+                               const float *g_mu, const float *g_var,
+                               void *grad_a, void *grad_p, void *grad_phi, void *grad_b,
+                               float *grad_lambda0, float *grad_eta0,
+                               int64_t B, int64_t T, int64_t H, int64_t N,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Which backward kernel kla_scan_backward would launch (only the alignment of
+ * a and p is looked at; outputs are assumed 16-byte aligned), written to
+ * *kernel: 1 = one thread per channel walking the sequence backwards (any
+ * shape), 2 = the channel-owning streaming kernel (16-byte aligned arrays,
+ * H*N*elem a multiple of 16 bytes, H*N >= 32); *launches = kernel launches
+ * per call (2 when a workspace clear precedes the streaming kernel).  0 and
+ * 0 for B*H*N == 0.  Honours kla_debug_force_backward_kernel.
+ */
+kla_status_t kla_scan_backward_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
+                                    const void *a, const void *p, int *kernel, int *launches);
+
+/*
+ * Test hook: which backward kernel later kla_scan_backward calls use.
+ * 0 (default): by shape; 1: one thread per channel; 2: the streaming kernel
+ * where its geometry holds.  Results agree to rounding.  KLA_ERR_INVALID_ARG
+ * for other values.
+ */
+kla_status_t kla_debug_force_backward_kernel(int which);
+
+/*
  * Synchronise `stream`, then report the first failure since the previous
  * call on the current device: KLA_ERR_CUDA for a CUDA error (sticky or not),
  * KLA_ERR_TIMEOUT if a kernel's bounded wait ran out (the outputs that
@@ -280,8 +359,11 @@ int kla_forward_chunk_tokens(void);
  * NaN and earlier tokens are unaffected.  In the chunked kernel a later chunk
  * is either exact (its look-back composed the stalled chunk's aggregate) or
  * NaN; in the streaming kernel every later token of the same channels is NaN
- * (the state is handed from chunk to chunk).  -1 (the default) turns the hook
- * off.
+ * (the state is handed from chunk to chunk).  The streaming backward kernel
+ * of kla_scan_backward honours it too: the carry into the backward chunk
+ * holding that token is poisoned, so the gradients of that chunk and of every
+ * earlier token of the same channels are NaN, later tokens are exact.  -1
+ * (the default) turns the hook off.
  */
 kla_status_t kla_debug_stall_chunk(int64_t chunk);
 

@@ -11,6 +11,8 @@ _API_NAMES = {
     "set_wait_limit_ns", "debug_unset_flag_wait", "debug_stall_chunk", "chunk_tokens",
     "debug_force_forward_kernel", "forward_plan", "host_workspace_size",
     "KlaError", "lib", "load_library", "scan_forward_static",
+    "scan_backward", "backward_workspace_size", "backward_plan", "debug_force_backward_kernel",
+    "KalmanFilterScan", "kalman_filter",
 }
 
 

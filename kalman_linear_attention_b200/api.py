@@ -51,6 +51,13 @@ SIGNATURES = {
                                                             ctypes.POINTER(_SZ)]),
     "kla_scan_forward_host": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP,
                                              _I64, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
+    "kla_scan_backward_workspace_size": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int,
+                                                        ctypes.POINTER(_SZ)]),
+    "kla_scan_backward": (ctypes.c_int, [_VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                         _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
+    "kla_scan_backward_plan": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP,
+                                              ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "kla_debug_force_backward_kernel": (ctypes.c_int, [ctypes.c_int]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -308,3 +315,108 @@ def scan_forward_static(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: 
             _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), B, T, H, N,
             _stream_handle(stream))
     _check(st, "kla_scan_forward_static")
+
+
+# ---------------------------------------------------------------- gradients
+def backward_workspace_size(B: int, T: int, H: int, N: int, dtype: torch.dtype = torch.float32) -> int:
+    code = KLA_BF16 if dtype == torch.bfloat16 else KLA_F32
+    out = ctypes.c_size_t(0)
+    _check(lib().kla_scan_backward_workspace_size(B, T, H, N, code, ctypes.byref(out)),
+           "kla_scan_backward_workspace_size")
+    return int(out.value)
+
+
+def backward_plan(a: torch.Tensor, p: torch.Tensor) -> Tuple[int, int]:
+    """(kernel, launches) that scan_backward would use: kernel 1 = one thread
+    per channel, 2 = channel-owning streaming kernel."""
+    B, T, H, N = a.shape
+    k, n = ctypes.c_int(0), ctypes.c_int(0)
+    with torch.cuda.device(a.device):
+        _check(lib().kla_scan_backward_plan(B, T, H, N, _dtype_code(a), _ptr(a), _ptr(p), ctypes.byref(k),
+                                            ctypes.byref(n)), "kla_scan_backward_plan")
+    return int(k.value), int(n.value)
+
+
+def debug_force_backward_kernel(which: int) -> None:
+    """0: choose by shape; 1: one thread per channel; 2: streaming kernel."""
+    _check(lib().kla_debug_force_backward_kernel(int(which)), "kla_debug_force_backward_kernel")
+
+
+def scan_backward(a: torch.Tensor, p: torch.Tensor, lam0: torch.Tensor, eta0: torch.Tensor,
+                  lam: torch.Tensor, eta: torch.Tensor,
+                  g_lam: Optional[torch.Tensor] = None, g_eta: Optional[torch.Tensor] = None,
+                  g_mu: Optional[torch.Tensor] = None, g_var: Optional[torch.Tensor] = None, *,
+                  want: Sequence[bool] = (True,) * 6,
+                  out: Optional[Sequence[Optional[torch.Tensor]]] = None,
+                  workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> Tuple[Optional[torch.Tensor], ...]:
+    """Gradients through scan_forward (kla_scan_backward).
+
+    ``a``, ``p`` are the forward inputs, ``lam0``, ``eta0`` its prior and
+    ``lam``, ``eta`` its outputs; ``g_*`` are the loss gradients with respect
+    to the four outputs (None = zero).  Returns the gradients with respect to
+    (a, p, phi, b, lam0, eta0): the first four in the inputs' dtype, the prior
+    ones fp32, None where ``want`` is False.  Enqueued on ``stream`` without
+    synchronising.
+    """
+    if a.dim() != 4 or a.shape != p.shape or a.dtype != p.dtype:
+        raise ValueError("a and p must share one [B, T, H, N] shape and dtype")
+    B, T, H, N = a.shape
+    if lam.shape != a.shape or eta.shape != a.shape:
+        raise ValueError("lam and eta must be the forward outputs, [B, T, H, N]")
+    if lam0.shape != (B, H, N) or eta0.shape != (B, H, N):
+        raise ValueError("lam0 and eta0 must be [B, H, N]")
+    grads_in = [g_lam, g_eta, g_mu, g_var]
+    for t in [lam, eta, lam0, eta0] + [g for g in grads_in if g is not None]:
+        if t.dtype != torch.float32:
+            raise TypeError("states, prior and output gradients must be float32")
+    for g in grads_in:
+        if g is not None and g.shape != a.shape:
+            raise ValueError("output gradients must be [B, T, H, N]")
+    _require_cuda(a, p, lam0, eta0, lam, eta, *grads_in)
+    code = _dtype_code(a)
+    dev = a.device
+    if out is None:
+        outs = [torch.empty((B, T, H, N), dtype=a.dtype, device=dev) if w else None for w in want[:4]]
+        outs += [torch.empty((B, H, N), dtype=torch.float32, device=dev) if w else None for w in want[4:6]]
+    else:
+        outs = list(out)
+        _require_cuda(*outs)
+    if workspace is None:
+        n = backward_workspace_size(B, T, H, N, a.dtype)
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    with torch.cuda.device(dev):
+        st = lib().kla_scan_backward(
+            _ptr(a), _ptr(p), code, _ptr(lam0), _ptr(eta0), _ptr(lam), _ptr(eta),
+            *[_ptr(g) for g in grads_in], *[_ptr(o) for o in outs], B, T, H, N,
+            _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream_handle(stream))
+    _check(st, "kla_scan_backward")
+    return tuple(outs)
+
+
+class KalmanFilterScan(torch.autograd.Function):
+    """Differentiable filter scan: forward = kla_scan_forward, backward =
+    kla_scan_backward.  Inputs (a, p, phi, b, lam0, eta0) as in scan_forward
+    (CUDA tensors); returns (lambda, eta, mu, var)."""
+
+    @staticmethod
+    def forward(ctx, a, p, phi, b, lam0, eta0):
+        ctx.set_materialize_grads(False)
+        lam, eta, mu, var = scan_forward(a, p, phi, b, lam0, eta0)
+        ctx.save_for_backward(a, p, lam0, eta0, lam, eta)
+        return lam, eta, mu, var
+
+    @staticmethod
+    def backward(ctx, g_lam, g_eta, g_mu, g_var):
+        a, p, lam0, eta0, lam, eta = ctx.saved_tensors
+        grads = [None if g is None else g.contiguous() for g in (g_lam, g_eta, g_mu, g_var)]
+        if all(g is None for g in grads):
+            return (None,) * 6
+        return scan_backward(a, p, lam0, eta0, lam, eta, *grads, want=ctx.needs_input_grad)
+
+
+def kalman_filter(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.Tensor,
+                  lam0: torch.Tensor, eta0: torch.Tensor):
+    """(lambda, eta, mu, var) of the filter, differentiable with respect to
+    every input through the CUDA backward scan."""
+    return KalmanFilterScan.apply(a, p, phi, b, lam0, eta0)

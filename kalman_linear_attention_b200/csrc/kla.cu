@@ -1,7 +1,8 @@
 // kla.cu -- host side of the C ABI declared in include/kla.h: argument
 // checks, workspace layout, TMA tensor maps and kernel launches.  Every step
-// of the filter runs in the kernels of kla_forward.cuh / kla_step.cuh; this
-// file only validates, describes memory and launches.
+// of the filter and of its gradients runs in the kernels of kla_forward.cuh,
+// kla_forward_stream.cuh, kla_step.cuh and kla_backward.cuh; this file only
+// validates, describes memory and launches.
 #include "kla.h"
 
 #include <cuda.h>
@@ -15,6 +16,7 @@
 #include <set>
 #include <utility>
 
+#include "kla_backward.cuh"
 #include "kla_forward.cuh"
 #include "kla_forward_stream.cuh"
 #include "kla_step.cuh"
@@ -677,4 +679,220 @@ KLA_API kla_status_t kla_scan_forward_static(const void *a, const void *p, const
     // (ticket counter and ready flags) on `stream` before its scan kernel.
     return kla_scan_forward(a, p, phi, b, in_dtype, lambda0, eta0, lambda_out, eta_out, mu_out,
                             var_out, B, T, H, N, scratch, (size_t)KLA_STATIC_SCRATCH_BYTES, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Gradients: kla_scan_backward (kernels in kla_backward.cuh).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Backward streaming kernel: chunk length (16 tokens: a chunk warp holds six
+// L-token arrays and two (L+1)-token arrays of its chunk in registers), chunk
+// warps and output group per dtype; the ring takes what shared memory is left.
+#ifndef KLA_BWD_L
+#define KLA_BWD_L 16
+#endif
+#ifndef KLA_BWD_W_F32
+#define KLA_BWD_W_F32 9
+#endif
+#ifndef KLA_BWD_W_BF16
+#define KLA_BWD_W_BF16 9
+#endif
+#ifndef KLA_BWD_G_F32
+#define KLA_BWD_G_F32 8
+#endif
+#ifndef KLA_BWD_G_BF16
+#define KLA_BWD_G_BF16 8
+#endif
+constexpr int kBL = KLA_BWD_L;
+template <typename Tin> constexpr int bwd_warps() { return sizeof(Tin) == 4 ? KLA_BWD_W_F32 : KLA_BWD_W_BF16; }
+template <typename Tin> constexpr int bwd_group() { return sizeof(Tin) == 4 ? KLA_BWD_G_F32 : KLA_BWD_G_BF16; }
+template <typename Tin>
+constexpr int bwd_stages() {
+    constexpr int W = bwd_warps<Tin>();
+    constexpr int G = bwd_group<Tin>();
+    const int stage = 2 * kBL * 32 * (int)sizeof(Tin) + 2 * (kBL + 1) * 32 * 4 + 4 * kBL * 32 * 4;
+    const int fixed = W * 2 * 4 * G * 32 * (int)sizeof(Tin) + W * 2 * 32 * 4 + W * 8 + 2048;
+    const int ns = (KLA_STREAM_SMEM - fixed) / stage;
+    return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
+}
+
+// 0: choose by shape; 1: the one-thread-per-channel kernel; 2: the streaming
+// kernel (test hook kla_debug_force_backward_kernel).
+std::atomic<int> g_force_bwd_kernel{0};
+
+// 2 when the streaming kernel's TMA geometry holds (16-byte aligned arrays,
+// H*N*elem a multiple of 16 bytes, H*N >= 32, T >= 1) and the tensor-map
+// encoder is available; 1 otherwise (or when forced).
+int backward_kernel_choice(int64_t T, int64_t HN, size_t esz, const void *const *ptrs, int nptrs) {
+    if (g_force_bwd_kernel.load() == 1 || T == 0) return 1;
+    bool ok = (HN * (int64_t)esz) % 16 == 0 && HN >= 32 && encode_fn() != nullptr;
+    for (int k = 0; k < nptrs && ok; ++k)
+        if (ptrs[k] && !aligned16(ptrs[k])) ok = false;
+    return ok ? 2 : 1;
+}
+
+template <typename Tin>
+cudaError_t launch_backward_stream(const kla::BwdParams &prm, const kla::BwdMaps &maps, cudaStream_t stream) {
+    constexpr int W = bwd_warps<Tin>();
+    constexpr int G = bwd_group<Tin>();
+    constexpr int NS = bwd_stages<Tin>();
+    using Cfg = kla::BwdTile<Tin, kBL, W, NS, G>;
+    static_assert(NS >= W && Cfg::SMEM <= 227 * 1024, "backward kernel shared memory");
+    auto kernel = kla::kla_backward_stream_kernel<Tin, kBL, W, NS, G>;
+    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
+    kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+unsigned bwd_stage_tx(unsigned g_mask) {
+    unsigned tx = 2u * kBL * 32u * (unsigned)sizeof(Tin) + 2u * (kBL + 1) * 32u * 4u;
+    for (int k = 0; k < 4; ++k)
+        if (g_mask >> k & 1u) tx += kBL * 32u * 4u;
+    return tx;
+}
+
+template <typename Tin>
+cudaError_t launch_backward_seq(const kla::BwdParams &prm, cudaStream_t stream) {
+    const int threads = 128;
+    const int64_t blocks = (prm.C + threads - 1) / threads;
+    kla::kla_backward_seq_kernel<Tin><<<(unsigned)blocks, threads, 0, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+KLA_API kla_status_t kla_scan_backward_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                                      kla_dtype_t in_dtype, size_t *bytes) {
+    if (!bytes || B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems)) return KLA_ERR_INVALID_ARG;
+    if (elems == 0) {
+        *bytes = 0;
+        return KLA_OK;
+    }
+    *bytes = stream_ws_layout(B * ((HN + 31) / 32), KLA_STREAM_MAX_PARTS).total;
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_scan_backward(const void *a, const void *p, kla_dtype_t in_dtype,
+                                       const float *lambda0, const float *eta0,
+                                       const float *lambda_out, const float *eta_out,
+                                       const float *g_lambda, const float *g_eta, const float *g_mu,
+                                       const float *g_var, void *grad_a, void *grad_p, void *grad_phi,
+                                       void *grad_b, float *grad_lambda0, float *grad_eta0,
+                                       int64_t B, int64_t T, int64_t H, int64_t N,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, C = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, HN, &C) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems))
+        return KLA_ERR_INVALID_ARG;
+    if (C == 0) return KLA_OK;
+    if (!lambda0 || !eta0) return KLA_ERR_INVALID_ARG;
+    if (elems > 0 && (!a || !p || !lambda_out || !eta_out)) return KLA_ERR_INVALID_ARG;
+    const size_t esz = dtype_size(in_dtype);
+    int64_t in_bytes = 0, f_bytes = 0, c_bytes = 0;
+    if (!mul_ok(elems, (int64_t)esz, &in_bytes) || !mul_ok(elems, 4, &f_bytes) || !mul_ok(C, 4, &c_bytes))
+        return KLA_ERR_INVALID_ARG;
+    const Range outs[6] = {range_of(grad_a, in_bytes), range_of(grad_p, in_bytes), range_of(grad_phi, in_bytes),
+                           range_of(grad_b, in_bytes), range_of(grad_lambda0, c_bytes),
+                           range_of(grad_eta0, c_bytes)};
+    const Range ins[11] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(lambda0, c_bytes),
+                           range_of(eta0, c_bytes), range_of(lambda_out, f_bytes), range_of(eta_out, f_bytes),
+                           range_of(g_lambda, f_bytes), range_of(g_eta, f_bytes), range_of(g_mu, f_bytes),
+                           range_of(g_var, f_bytes), range_of(workspace, (int64_t)workspace_bytes)};
+    if (any_overlap(outs, 6, ins, 11)) return KLA_ERR_INVALID_ARG;
+    size_t need = 0;
+    if (kla_scan_backward_workspace_size(B, T, H, N, in_dtype, &need) != KLA_OK) return KLA_ERR_INVALID_ARG;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KLA_ERR_WORKSPACE_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KLA_ERR_MISALIGNED;
+    if (T > INT32_MAX - 1 || HN > INT32_MAX || B > INT32_MAX) return KLA_ERR_INVALID_ARG;
+
+    kla::BwdParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.a = a; prm.p = p; prm.lam = lambda_out; prm.eta = eta_out;
+    prm.g[0] = g_lambda; prm.g[1] = g_eta; prm.g[2] = g_mu; prm.g[3] = g_var;
+    prm.grad[0] = grad_a; prm.grad[1] = grad_p; prm.grad[2] = grad_phi; prm.grad[3] = grad_b;
+    prm.lam0 = lambda0; prm.eta0 = eta0; prm.g_lam0 = grad_lambda0; prm.g_eta0 = grad_eta0;
+    prm.T = T; prm.HN = HN; prm.C = C;
+    prm.wait_ns = g_wait_ns.load();
+    prm.stall_chunk = -1;
+    for (int k = 0; k < 4; ++k) {
+        if (prm.g[k]) prm.g_mask |= 1u << k;
+        if (prm.grad[k]) prm.grad_mask |= 1u << k;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const void *ptrs[14] = {a, p, lambda_out, eta_out, g_lambda, g_eta, g_mu, g_var,
+                            grad_a, grad_p, grad_phi, grad_b, nullptr, nullptr};
+
+    if (backward_kernel_choice(T, HN, esz, ptrs, 12) == 2) {
+        const CUtensorMapDataType tdt =
+            in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        const int G = in_dtype == KLA_F32 ? bwd_group<float>() : bwd_group<__nv_bfloat16>();
+        kla::BwdMaps maps;
+        std::memset(&maps, 0, sizeof(maps));
+        bool ok = encode_stream_map(&maps.in[0], a, tdt, esz, B, T, HN, kBL) &&
+                  encode_stream_map(&maps.in[1], p, tdt, esz, B, T, HN, kBL) &&
+                  encode_stream_map(&maps.in[2], lambda_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN, kBL + 1) &&
+                  encode_stream_map(&maps.in[3], eta_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN, kBL + 1);
+        for (int k = 0; k < 4 && ok; ++k)
+            if (prm.g[k])
+                ok = encode_stream_map(&maps.in[4 + k], prm.g[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN, kBL);
+        for (int k = 0; k < 4 && ok; ++k)
+            if (prm.grad[k]) ok = encode_stream_map(&maps.out[k], prm.grad[k], tdt, esz, B, T, HN, G);
+        if (ok) {
+            prm.ntiles = B * ((HN + 31) / 32);
+            prm.nct = (int)((HN + 31) / 32);
+            prm.nchunks = (int)((T + kBL - 1) / kBL);
+            prm.stage_tx = in_dtype == KLA_F32 ? bwd_stage_tx<float>(prm.g_mask)
+                                               : bwd_stage_tx<__nv_bfloat16>(prm.g_mask);
+            prm.stall_chunk = g_stall_chunk.load() >= 0 ? g_stall_chunk.load() * kL / kBL : -1;
+            prm.parts = stream_parts(prm.ntiles, prm.nchunks);
+            prm.chunks_per_part = (prm.nchunks + prm.parts - 1) / prm.parts;
+            prm.nunits = prm.ntiles * prm.parts;
+            unsigned char *ws = static_cast<unsigned char *>(workspace);
+            prm.ticket = reinterpret_cast<unsigned *>(ws);
+            if (prm.parts > 1) {
+                const StreamWs sw = stream_ws_layout(prm.ntiles, prm.parts);
+                prm.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
+                prm.part_state = reinterpret_cast<float *>(ws + sw.state_off);
+                if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
+            }
+            const cudaError_t e = in_dtype == KLA_F32 ? launch_backward_stream<float>(prm, maps, st)
+                                                      : launch_backward_stream<__nv_bfloat16>(prm, maps, st);
+            return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+        }
+    }
+    const cudaError_t e = in_dtype == KLA_F32 ? launch_backward_seq<float>(prm, st)
+                                              : launch_backward_seq<__nv_bfloat16>(prm, st);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+KLA_API kla_status_t kla_scan_backward_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
+                                            const void *a, const void *p, int *kernel, int *launches) {
+    if (!kernel || !launches || B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, C = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, HN, &C)) return KLA_ERR_INVALID_ARG;
+    if (C == 0) {
+        *kernel = 0;
+        *launches = 0;
+        return KLA_OK;
+    }
+    const void *ptrs[2] = {a, p};
+    *kernel = backward_kernel_choice(T, HN, dtype_size(in_dtype), ptrs, 2);
+    *launches = 1;
+    if (*kernel == 2 && stream_parts(B * ((HN + 31) / 32), (T + kBL - 1) / kBL) > 1) *launches = 2;
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_debug_force_backward_kernel(int which) {
+    if (which < 0 || which > 2) return KLA_ERR_INVALID_ARG;
+    g_force_bwd_kernel.store(which);
+    return KLA_OK;
 }

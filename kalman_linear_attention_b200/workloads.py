@@ -28,6 +28,7 @@ sigmoid(x) = 1/(1+e^-x); all evaluated in fp64):
 from __future__ import annotations
 
 import dataclasses
+import re
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 from typing import Dict, Iterator, Tuple
@@ -59,7 +60,16 @@ class Workload:
         return self.B * self.T * self.H * self.N
 
     def with_shape(self, **kw) -> "Workload":
-        return dataclasses.replace(self, **kw)
+        """The same distributions and seed at another shape; the summary
+        names the new sizes."""
+        summary = self.summary
+        for k, v in kw.items():
+            if k in ("B", "H", "N"):
+                summary = re.sub(rf"\b{k}=\d+", f"{k}={v}", summary)
+            elif k == "T":
+                summary = re.sub(r"\bT=\d+", f"T={v}", summary)
+                summary = re.sub(r"\b\d+ one-token steps", f"{v} one-token steps", summary)
+        return dataclasses.replace(self, summary=summary, **kw)
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -180,6 +190,50 @@ def generate(w: Workload) -> Dict[str, np.ndarray]:
 def prior(w: Workload) -> Dict[str, np.ndarray]:
     return {"lam0": np.ones((w.B, w.H, w.N), dtype=np.float32),
             "eta0": np.zeros((w.B, w.H, w.N), dtype=np.float32)}
+
+
+def random_prior(w: Workload, seed: int = 777) -> Dict[str, np.ndarray]:
+    """A non-trivial prior: lam0 ~ logU(0.1, 10), eta0 ~ N(0, 1), fp32 [B, H, N]."""
+    rng = np.random.default_rng([w.seed, seed])
+    n = w.B * w.H * w.N
+    return {"lam0": _log_uniform(rng, 0.1, 10.0, n).astype(np.float32).reshape(w.B, w.H, w.N),
+            "eta0": rng.standard_normal(n).astype(np.float32).reshape(w.B, w.H, w.N)}
+
+
+# Loss gradients with respect to the four outputs (lambda, eta, mu, var), the
+# inputs of the backward scan: standard normal fp32, i.e. the gradients of a
+# random linear loss.  Their streams are spawned from (seed, 1), independent
+# of the forward inputs' streams.
+GRAD_NAMES = ("g_lam", "g_eta", "g_mu", "g_var")
+
+
+def iter_output_grad_rows(w: Workload, rows_per_block: int | None = None
+                          ) -> Iterator[Tuple[int, int, Dict[str, np.ndarray]]]:
+    """Like iter_rows, for the four output gradients."""
+    HN = w.H * w.N
+    rows = w.B * w.T
+    if rows_per_block is None:
+        rows_per_block = max(1, _BLOCK_ELEMS // max(HN, 1))
+    children = np.random.SeedSequence([w.seed, 1]).spawn(len(GRAD_NAMES))
+    rngs = [np.random.Generator(np.random.PCG64(c)) for c in children]
+    with ThreadPoolExecutor(max_workers=len(GRAD_NAMES)) as pool:
+        r0 = 0
+        while r0 < rows:
+            r1 = min(rows, r0 + rows_per_block)
+            n = (r1 - r0) * HN
+            futs = [pool.submit(lambda g, m: g.standard_normal(m, dtype=np.float32), rng, n) for rng in rngs]
+            yield r0, r1, {k: f.result().reshape(r1 - r0, w.H, w.N) for k, f in zip(GRAD_NAMES, futs)}
+            r0 = r1
+
+
+def generate_output_grads(w: Workload) -> Dict[str, np.ndarray]:
+    """All four output gradients of a workload, fp32 [B, T, H, N]."""
+    full = {k: np.empty((w.B * w.T, w.H, w.N), dtype=np.float32) for k in GRAD_NAMES}
+    if w.B * w.T * w.H * w.N:
+        for r0, r1, blk in iter_output_grad_rows(w):
+            for k in GRAD_NAMES:
+                full[k][r0:r1] = blk[k]
+    return {k: v.reshape(w.B, w.T, w.H, w.N) for k, v in full.items()}
 
 
 def channel_sample(w: Workload, count: int, seed: int = 12345) -> np.ndarray:

@@ -121,3 +121,42 @@ def test_host_workspace_size(lib):
     assert lib.kla_scan_forward_host_workspace_size(1, 0, 1, 1, 0, 0, ctypes.byref(out)) == 0 and out.value == 0
     assert lib.kla_scan_forward_host_workspace_size(1, 10, 1, 1, 0, -1, ctypes.byref(out)) == 1
     assert lib.kla_scan_forward_host_workspace_size(1, 10, 1, 1, 4, 0, ctypes.byref(out)) == 2
+
+
+def test_backward_host_argument_errors(lib):
+    """kla_scan_backward: the same host-side checks, before any CUDA call."""
+    bwd = lib.kla_scan_backward
+    P = 1 << 20  # fake, never dereferenced
+    names = ["a", "p", "dt", "lam0", "eta0", "lam", "eta", "gl", "ge", "gm", "gv",
+             "ga", "gp", "gphi", "gb", "glam0", "geta0", "B", "T", "H", "N", "ws", "wsb", "stream"]
+    base = dict(a=P, p=2 * P, dt=0, lam0=3 * P, eta0=4 * P, lam=5 * P, eta=6 * P, gl=7 * P, ge=None,
+                gm=8 * P, gv=None, ga=9 * P, gp=10 * P, gphi=11 * P, gb=12 * P, glam0=13 * P,
+                geta0=14 * P, B=1, T=4, H=1, N=4, ws=16 * P, wsb=1 << 20, stream=None)
+    args = lambda **kw: [kw.get(n, base[n]) for n in names]
+    assert bwd(*args(H=-1)) == 1
+    assert bwd(*args(dt=2)) == 2
+    assert bwd(*args(a=None)) == 1
+    assert bwd(*args(lam=None)) == 1
+    assert bwd(*args(lam0=None)) == 1
+    assert bwd(*args(gp=9 * P)) == 1              # grad_p overlaps grad_a
+    assert bwd(*args(gb=5 * P)) == 1              # grad_b overlaps lambda_out
+    assert bwd(*args(glam0=7 * P)) == 1           # prior gradient overlaps g_lambda
+    assert bwd(*args(ga=16 * P)) == 1             # overlaps the workspace
+    assert bwd(*args(wsb=16)) == 3
+    assert bwd(*args(ws=None, wsb=0)) == 3
+    assert bwd(*args(ws=16 * P + 8)) == 6
+    assert bwd(*args(B=0, a=None, lam0=None)) == 0  # no channels: nothing enqueued
+    out = ctypes.c_size_t(7)
+    assert lib.kla_scan_backward_workspace_size(1, 0, 32, 128, 0, ctypes.byref(out)) == 0 and out.value == 0
+    assert lib.kla_scan_backward_workspace_size(1, 65536, 32, 128, 1, ctypes.byref(out)) == 0
+    # run-boundary carries: at most 3 boundaries x 64 floats per 32-channel tile, plus flags
+    assert 128 * 3 * 64 * 4 <= out.value <= 128 * 3 * 64 * 4 + 128 * 3 * 4 + 4096
+    assert lib.kla_scan_backward_workspace_size(1, 1, 1, 1, 3, ctypes.byref(out)) == 2
+    k, n = ctypes.c_int(-1), ctypes.c_int(-1)
+    assert lib.kla_scan_backward_plan(0, 5, 1, 1, 0, P, P, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) == (0, 0)
+    assert lib.kla_scan_backward_plan(1, 64, 1, 7, 0, P, P, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) == (1, 1)                      # H*N = 7: one thread per channel
+    assert lib.kla_scan_backward_plan(1, 64, 32, 128, 0, P + 4, P, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert k.value == 1                                       # unaligned input
+    assert lib.kla_debug_force_backward_kernel(3) == 1
