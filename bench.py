@@ -232,7 +232,7 @@ def backward_bytes_per_tc(w: wl.Workload) -> int:
     return 2 * e + 2 * 4 + 4 * 4 + 4 * e
 
 
-def time_backward(kla, w, dev, outs, steps: int, warmup: int, peak: float):
+def time_backward(kla, w, dev, outs, steps: int, warmup: int, peak: float, traffic_key: str):
     """kla_scan_backward on the forward's lambda / eta with all four output
     gradients present (the general case), CUDA events per launch."""
     import torch
@@ -272,7 +272,8 @@ def time_backward(kla, w, dev, outs, steps: int, warmup: int, peak: float):
                        2: "kla_backward_stream_kernel (channel-owning streaming, reverse time)"}[plan[0]],
             "gpu_launches": plan[1] * steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "algorithmic_bytes_per_launch": bpt * tc, "traffic": None},
+                         "algorithmic_bytes_per_launch": bpt * tc,
+                         "traffic": recorded_traffic(traffic_key, plan[0])},
             "data": "forward outputs of the timed forward; output gradients from a seeded torch.randn on the device"}
 
 
@@ -408,7 +409,9 @@ def run_ours(args):
 
     backward = None
     if not args.no_backward:
-        backward = time_backward(kla, w, dev, fwd_outs, args.backward_steps, args.warmup, peak)
+        backward = time_backward(kla, w, dev, fwd_outs, args.backward_steps, args.warmup, peak,
+                                 (args.workload if not args.tokens else f"{args.workload}@T={args.tokens}")
+                                 + ":backward")
     del fwd_outs
 
     e2e = None

@@ -60,12 +60,13 @@ static_assert(kCkpt >= 1 && kCkpt <= 32, "checkpoint interval must be 1..32");
 #ifndef KLA_STREAM_L
 #define KLA_STREAM_L 32
 #endif
-// Chunk warps: fp32 stages are 16 KB, so 9 warps leave two ring stages free
-// for prefetch; bf16 stages are 8 KB and the ring is deep anyway, so 11
-// (12 warps in all = 3 per SM sub-partition, the most that still allows 168
-// registers per thread).
+// Chunk warps: 6 for fp32 (7 warps in all, up to 255 registers per thread,
+// a 10-stage ring of 16 KB stages); measured on the long workload against 5,
+// 7 and 9 chunk warps on the same GPU: 6 was 3-7% faster than each.  bf16
+// stages are 8 KB and the ring is deep anyway, so 11 (12 warps in all = 3 per
+// SM sub-partition, the most that still allows 168 registers per thread).
 #ifndef KLA_STREAM_W_F32
-#define KLA_STREAM_W_F32 9
+#define KLA_STREAM_W_F32 6
 #endif
 #ifndef KLA_STREAM_W_BF16
 #define KLA_STREAM_W_BF16 11
@@ -692,11 +693,15 @@ namespace {
 #ifndef KLA_BWD_L
 #define KLA_BWD_L 16
 #endif
+// 6 (fp32) and 7 (bf16) chunk warps, at up to 210 registers per thread:
+// same-GPU sweeps over 4-9 warps and 4-16 token output groups put these
+// first (fp32 long workload 96-97% of the copy bandwidth; 9 warps, capped at
+// 168 registers and spilling, 90%).
 #ifndef KLA_BWD_W_F32
-#define KLA_BWD_W_F32 9
+#define KLA_BWD_W_F32 6
 #endif
 #ifndef KLA_BWD_W_BF16
-#define KLA_BWD_W_BF16 9
+#define KLA_BWD_W_BF16 7
 #endif
 #ifndef KLA_BWD_G_F32
 #define KLA_BWD_G_F32 8

@@ -119,6 +119,16 @@ struct BwdParams {
     int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
 };
 
+// What the producer tells the chunk warps about the chunk in a stage
+// (computed once per work unit, so the chunk warps do no index division).
+struct BwdChunk {
+    int64_t tile;      // b * nct + channel tile
+    int chunk;         // chunk index in the sequence; -1: no more work
+    int run;           // the run of the tile this chunk belongs to
+    int bb, ct;        // batch row, 32-channel tile within the row
+    int run_lo, run_hi;  // first and last chunk of the run
+};
+
 struct BwdMaps {
     CUtensorMap in[8];   // a, p (input dtype), lambda, eta (box L + 1 rows), g_lambda, g_eta, g_mu, g_var
     CUtensorMap out[4];  // d/d a, p, phi, b (input dtype), box G rows
@@ -146,8 +156,8 @@ struct BwdTile {
     static_assert(OUTBOX_BYTES % 128 == 0, "TMA store sources stay 128-byte aligned");
     static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][32]
     static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][32] fp32
-    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: unit, chunk
-    static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128);
+    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // [NS] BwdChunk
+    static constexpr int BAR_OFF = align_up(META_OFF + NS * (int)sizeof(BwdChunk), 128);
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
 
@@ -161,8 +171,7 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
     uint64_t *empty = full + NS;
     uint64_t *carry_bar = empty + NS;
     float *slots = reinterpret_cast<float *>(smem + Cfg::CARRY_OFF);
-    int64_t *meta_unit = reinterpret_cast<int64_t *>(smem + Cfg::META_OFF);  // -1: no more work
-    int64_t *meta_chunk = meta_unit + NS;
+    BwdChunk *meta = reinterpret_cast<BwdChunk *>(smem + Cfg::META_OFF);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -189,21 +198,22 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane != 0) return;
-        int64_t seq = 0;
+        int next = 0, round = 0;  // next stage to fill; completed passes over the ring
         auto claim = [&]() -> int {
-            const int s = (int)(seq % NS);
-            if (seq >= NS) mbar_wait_or_flag(&empty[s], (unsigned)((seq / NS - 1) & 1), prm.wait_ns);
-            ++seq;
+            const int s = next;
+            if (round > 0) mbar_wait_or_flag(&empty[s], (unsigned)((round - 1) & 1), prm.wait_ns);
+            if (++next == NS) {
+                next = 0;
+                ++round;
+            }
             return s;
         };
-        auto load = [&](int64_t unit, int64_t chunk) {
+        auto load = [&](const BwdChunk &m) {
             const int s = claim();
-            const int64_t tile = unit % prm.ntiles;
-            const int bb = (int)(tile / prm.nct);
-            const int x = (int)(tile - (int64_t)bb * prm.nct) * 32;
-            const int y = (int)(chunk * L);
-            meta_unit[s] = unit;
-            meta_chunk[s] = chunk;
+            const int x = m.ct * 32;
+            const int y = m.chunk * L;
+            const int bb = m.bb;
+            meta[s] = m;
             unsigned char *stage = smem + s * Cfg::STAGE_BYTES;
             mbar_arrive_expect_tx(&full[s], prm.stage_tx);
             tma_load_3d(stage, &maps.in[0], x, y, bb, &full[s]);
@@ -217,28 +227,36 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
                 if (prm.g_mask >> k & 1u)
                     tma_load_3d(stage + Cfg::OFF_G + k * Cfg::GR_BYTES, &maps.in[4 + k], x, y, bb, &full[s]);
         };
+        // one unit: the tile's run r, latest chunk first
+        auto unit_chunks = [&](int64_t u) {
+            BwdChunk m;
+            m.tile = u % prm.ntiles;
+            m.run = prm.parts - 1 - (int)(u / prm.ntiles);
+            m.bb = (int)(m.tile / prm.nct);
+            m.ct = (int)(m.tile - (int64_t)m.bb * prm.nct);
+            m.run_lo = m.run * prm.chunks_per_part;
+            m.run_hi = min(m.run_lo + prm.chunks_per_part, prm.nchunks) - 1;
+#pragma unroll 1
+            for (int c = m.run_hi; c >= m.run_lo; --c) {
+                m.chunk = c;
+                load(m);
+            }
+        };
         if (prm.parts == 1) {
 #pragma unroll 1
-            for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x)
-#pragma unroll 1
-                for (int64_t c = prm.nchunks - 1; c >= 0; --c) load(u, c);
+            for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
         } else {
 #pragma unroll 1
             for (;;) {
                 const int64_t u = (int64_t)atomicAdd(prm.ticket, 1u);
                 if (u >= prm.nunits) break;
-                const int64_t r = prm.parts - 1 - u / prm.ntiles;
-                const int64_t c0 = r * prm.chunks_per_part;
-                const int64_t c1 = c0 + prm.chunks_per_part < prm.nchunks ? c0 + prm.chunks_per_part
-                                                                          : (int64_t)prm.nchunks;
-#pragma unroll 1
-                for (int64_t c = c1 - 1; c >= c0; --c) load(u, c);
+                unit_chunks(u);
             }
         }
 #pragma unroll 1
         for (int k = 0; k < W; ++k) {
             const int s = claim();
-            meta_unit[s] = -1;
+            meta[s].chunk = -1;
             mbar_arrive(&full[s]);
         }
         return;
@@ -248,42 +266,56 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
     const int w = warp - 1;
     Tin *outbuf0 = reinterpret_cast<Tin *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
     int group_seq = 0;
+    // This warp takes the CTA's chunks j = w, w + W, w + 2W, ...: chunk j sits
+    // in stage j % NS (phase parity (j / NS) & 1), and its carry comes from
+    // warp (j - 1) % W.  Tracked incrementally (W <= NS).
+    int s = w;
+    unsigned par = 0;
+    const int prev_w = w > 0 ? w - 1 : W - 1;
 #pragma unroll 1
-    for (int64_t j = w;; j += W) {
-        const int s = (int)(j % NS);
-        mbar_wait_or_flag(&full[s], (unsigned)((j / NS) & 1), prm.wait_ns);
-        const int64_t unit = meta_unit[s];
-        if (unit < 0) break;
-        const int64_t chunk = meta_chunk[s];
-        const int64_t tile = unit % prm.ntiles;
-        const int64_t run = prm.parts - 1 - unit / prm.ntiles;
-        const int64_t bb = tile / prm.nct;
-        const int64_t ct = tile - bb * prm.nct;
-        const int64_t t0 = chunk * L;
+    for (int k = 0;; ++k) {
+        mbar_wait_or_flag(&full[s], par, prm.wait_ns);
+        const BwdChunk m = meta[s];
+        const int stage_s = s;
+        s += W;
+        if (s >= NS) {
+            s -= NS;
+            par ^= 1u;
+        }
+        if (m.chunk < 0) break;
+        const bool has_prev = k > 0 || w > 0;                  // j > 0
+        const unsigned prev_par = (unsigned)((w > 0 ? k : k - 1) & 1);  // ((j - 1) / W) & 1
+        const int chunk = m.chunk;
+        const int run = m.run;
+        const int64_t tile = m.tile;
+        const int64_t bb = m.bb;
+        const int64_t ct = m.ct;
+        const int64_t t0 = (int64_t)chunk * L;
         const int t_valid = (int)(prm.T - t0 < (int64_t)L ? prm.T - t0 : (int64_t)L);
         const int64_t ch = ct * 32 + lane;
         const bool cvalid = ch < prm.HN;
-        const unsigned char *stage = smem + s * Cfg::STAGE_BYTES;
+        const unsigned char *stage = smem + stage_s * Cfg::STAGE_BYTES;
         const Tin *sa = reinterpret_cast<const Tin *>(stage);
         const Tin *sp = reinterpret_cast<const Tin *>(stage + Cfg::OFF_P);
         const float *sl = reinterpret_cast<const float *>(stage + Cfg::OFF_LAM);  // row 0 = history
         const float *se = reinterpret_cast<const float *>(stage + Cfg::OFF_ETA);
         const float *sg = reinterpret_cast<const float *>(stage + Cfg::OFF_G);
-        const int64_t run_lo = run * prm.chunks_per_part;
-        const int64_t run_hi = (run_lo + prm.chunks_per_part < prm.nchunks ? run_lo + prm.chunks_per_part
-                                                                           : (int64_t)prm.nchunks) - 1;
-        const float prior_lam = (chunk == 0 && cvalid) ? prm.lam0[bb * prm.HN + ch] : 1.f;
-        const float prior_eta = (chunk == 0 && cvalid) ? prm.eta0[bb * prm.HN + ch] : 0.f;
+        const int run_lo = m.run_lo;
+        const int run_hi = m.run_hi;
+        float prior_lam = 1.f, prior_eta = 0.f;
+        if (chunk == 0 && cvalid) {
+            prior_lam = prm.lam0[bb * prm.HN + ch];
+            prior_eta = prm.eta0[bb * prm.HN + ch];
+        }
 
         // Carry entering the chunk from the later tokens: from the warp of
         // the later chunk, zero after the last chunk, or published by the
         // tile's later run at a run's last chunk.
         auto carry_in = [&](float &cE, float &cL) {
-            if (j > 0) {
-                const int ps = (int)((j - 1) % W);
-                mbar_wait_or_flag(&carry_bar[ps], (unsigned)(((j - 1) / W) & 1), prm.wait_ns);
-                cE = slots[ps * 64 + lane];
-                cL = slots[ps * 64 + 32 + lane];
+            if (has_prev) {
+                mbar_wait_or_flag(&carry_bar[prev_w], prev_par, prm.wait_ns);
+                cE = slots[prev_w * 64 + lane];
+                cL = slots[prev_w * 64 + 32 + lane];
             }
             if (chunk == prm.stall_chunk &&
                 !warp_wait_flags(lane == 0 ? &g_never_set_word : nullptr, prm.wait_ns)) {
@@ -307,11 +339,10 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
         };
         // Carry leaving the chunk towards the earlier tokens.
         auto carry_out = [&](float oE, float oL) {
-            const int ms = (int)(j % W);
-            slots[ms * 64 + lane] = oE;
-            slots[ms * 64 + 32 + lane] = oL;
+            slots[w * 64 + lane] = oE;
+            slots[w * 64 + 32 + lane] = oL;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&carry_bar[ms]);
+            if (lane == 0) mbar_arrive(&carry_bar[w]);
             if (chunk == run_lo && run > 0) {
                 const int64_t slot = tile * (prm.parts - 1) + (run - 1);
                 prm.part_state[slot * 64 + lane] = oE;
@@ -372,7 +403,7 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
                                  xgl[t], xge[t]);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&empty[stage_s]);
             if (chunk == 0) {
                 xl[0] = prior_lam;
                 xe[0] = prior_eta;
@@ -439,7 +470,7 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
                 group_end(buf, q);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&empty[stage_s]);
             carry_out(cE, cL);
             prior_out(cE, cL);
         }

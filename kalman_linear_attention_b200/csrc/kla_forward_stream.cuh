@@ -136,41 +136,47 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane != 0) return;
-        int64_t seq = 0;  // chunks (and end markers) handed to the chunk warps
+        int next = 0, round = 0;  // next stage to fill; completed passes over the ring
         auto claim = [&]() -> int {
-            const int s = (int)(seq % NS);
-            if (seq >= NS) mbar_wait_or_flag(&empty[s], (unsigned)((seq / NS - 1) & 1), prm.wait_ns);
-            ++seq;
+            const int s = next;
+            if (round > 0) mbar_wait_or_flag(&empty[s], (unsigned)((round - 1) & 1), prm.wait_ns);
+            if (++next == NS) {
+                next = 0;
+                ++round;
+            }
             return s;
         };
-        auto load = [&](int64_t unit, int64_t chunk) {
+        auto load = [&](int64_t unit, int chunk, int bb, int ct) {
             const int s = claim();
-            const int64_t tile = unit % prm.ntiles;
-            const int bb = (int)(tile / prm.nct);
-            const int ct = (int)(tile - (int64_t)bb * prm.nct);
             meta_unit[s] = unit;
             meta_chunk[s] = chunk;
             Tin *stage = reinterpret_cast<Tin *>(smem + s * Cfg::STAGE_BYTES);
             mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, (int)(chunk * L), bb, &full[s]);
+                tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, chunk * L, bb, &full[s]);
+        };
+        // one unit: the tile's run u / ntiles, in time order (its tile
+        // coordinates computed once per unit, not per chunk)
+        auto unit_chunks = [&](int64_t u) {
+            const int64_t tile = u % prm.ntiles;
+            const int part = (int)(u / prm.ntiles);
+            const int bb = (int)(tile / prm.nct);
+            const int ct = (int)(tile - (int64_t)bb * prm.nct);
+            const int first = part * prm.chunks_per_part;
+            const int last = min(first + prm.chunks_per_part, prm.nchunks) - 1;
+#pragma unroll 1
+            for (int c = first; c <= last; ++c) load(u, c, bb, ct);
         };
         if (prm.parts == 1) {
 #pragma unroll 1
-            for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x)
-#pragma unroll 1
-                for (int64_t c = 0; c < prm.nchunks; ++c) load(u, c);
+            for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
         } else {
 #pragma unroll 1
             for (;;) {
                 const int64_t u = (int64_t)atomicAdd(prm.ticket, 1u);
                 if (u >= prm.nunits) break;
-                const int64_t c0 = (u / prm.ntiles) * prm.chunks_per_part;
-                const int64_t c1 = c0 + prm.chunks_per_part < prm.nchunks ? c0 + prm.chunks_per_part
-                                                                          : (int64_t)prm.nchunks;
-#pragma unroll 1
-                for (int64_t c = c0; c < c1; ++c) load(u, c);
+                unit_chunks(u);
             }
         }
         // one end marker for each chunk warp

@@ -85,3 +85,41 @@ def test_stalled_chunk_in_streaming_kernel(kla):
     assert kla.get_error() == 0
     got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out2)}
     parity.assert_parity(got, ref, 1e-5, time_axis=1)
+
+
+def test_stalled_chunk_in_backward_kernel(kla):
+    """The streaming backward kernel hands the gradient carry from the later
+    chunk to the earlier one: a carry wait that runs out poisons that chunk's
+    gradients and those of every earlier token of its channels, leaves later
+    tokens exact, reports KLA_ERR_TIMEOUT, and the context stays usable."""
+    import test_backward_gpu as tb
+    kla.debug_force_backward_kernel(2)
+    try:
+        w = wl.WORKLOADS["tiny"].with_shape(B=2, T=512, H=2, N=64)
+        x = wl.generate(w)
+        go = wl.generate_output_grads(w)
+        d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
+        g = [torch.from_numpy(go[k]).to(DEV) for k in wl.GRAD_NAMES]
+        lam, eta, _, _ = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+        assert kla.get_error() == 0
+        kla.debug_stall_chunk(3)  # the backward chunk holding token 3 * chunk_tokens()
+        out = kla.scan_backward(d["a"], d["p"], d["lam0"], d["eta0"], lam, eta, *g)
+        assert kla.get_error() == 5
+        kla.debug_stall_chunk(-1)
+        stalled = 3 * kla.chunk_tokens()
+        ref = oracle.backward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"],
+                              *(go[k] for k in wl.GRAD_NAMES))
+        got = [o.double().cpu().numpy() for o in out]
+        # the chunk holding the stalled token ends at most 16 tokens later
+        exact_from = stalled + 16
+        later = {k: got[i][:, exact_from:] for i, k in enumerate(tb.GRADS)}
+        tb.assert_grad_parity(later, {k: ref[k][:, exact_from:] for k in tb.GRADS}, 1e-5, "after the stall")
+        for i in range(4):
+            assert np.isnan(got[i][:, :stalled + 1]).all()
+        assert np.isnan(got[4]).all() and np.isnan(got[5]).all()
+        out2 = kla.scan_backward(d["a"], d["p"], d["lam0"], d["eta0"], lam, eta, *g)
+        assert kla.get_error() == 0
+        got2 = {k: o.double().cpu().numpy() for k, o in zip(tb.GRADS + ("lam0", "eta0"), out2)}
+        tb.assert_grad_parity(got2, ref, 1e-5, "after recovery")
+    finally:
+        kla.debug_force_backward_kernel(0)
