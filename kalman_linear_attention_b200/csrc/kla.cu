@@ -62,22 +62,23 @@ static_assert(kCkpt >= 1 && kCkpt <= 32, "checkpoint interval must be 1..32");
 #endif
 // Chunk warps: 6 for fp32 (7 warps in all, up to 255 registers per thread,
 // a 10-stage ring of 16 KB stages); measured on the long workload against 5,
-// 7 and 9 chunk warps on the same GPU: 6 was 3-7% faster than each.  bf16
-// stages are 8 KB and the ring is deep anyway, so 11 (12 warps in all = 3 per
-// SM sub-partition, the most that still allows 168 registers per thread).
+// 7 and 9 chunk warps on the same GPU: 6 was 3-7% faster than each.  7 for
+// bf16 (8 KB stages, a 21-stage ring): on the LM-layer shape 2.7% faster than
+// 11 warps at 168 registers, and 6 or 8 were slower.
 #ifndef KLA_STREAM_W_F32
 #define KLA_STREAM_W_F32 6
 #endif
 #ifndef KLA_STREAM_W_BF16
-#define KLA_STREAM_W_BF16 11
+#define KLA_STREAM_W_BF16 7
 #endif
-// Tokens per output box (one TMA store per output per box): 8 for fp32
-// (measured 4-6% faster than 4 on the long workload, same-box A/B).
+// Tokens per output box (one TMA store per output per box): 8 (measured 4-6%
+// faster than 4 on the long workload, and with 7 bf16 chunk warps 18% faster
+// than 4 on the LM-layer shape; same-box A/B).
 #ifndef KLA_STREAM_G_F32
 #define KLA_STREAM_G_F32 8
 #endif
 #ifndef KLA_STREAM_G_BF16
-#define KLA_STREAM_G_BF16 4
+#define KLA_STREAM_G_BF16 8
 #endif
 #ifndef KLA_STREAM_SMEM
 #define KLA_STREAM_SMEM (227 * 1024)
