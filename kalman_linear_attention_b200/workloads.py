@@ -245,3 +245,68 @@ def channel_sample(w: Workload, count: int, seed: int = 12345) -> np.ndarray:
     # always include the first and last channel (tile edges)
     idx = np.unique(np.concatenate([idx, [0, C - 1]]))
     return idx
+
+
+# --------------------------------------------------------------------------
+# The fused KLA layer: per-token operators and values of H heads, per-channel
+# time-invariant decay and process noise over H x D x Ns state channels.
+@dataclass(frozen=True)
+class LayerWorkload:
+    name: str
+    B: int
+    T: int
+    H: int
+    D: int          # value dimension per head
+    Ns: int         # state expansion: state channels per value coordinate
+    dtype: str      # "f32" or "bf16": dtype of k, q, v, w on the device
+    seed: int
+    summary: str = ""
+
+    @property
+    def channels(self) -> int:
+        return self.B * self.H * self.D * self.Ns
+
+    @property
+    def token_channels(self) -> int:
+        return self.T * self.channels
+
+    def with_shape(self, **kw) -> "LayerWorkload":
+        summary = self.summary
+        for k, v in kw.items():
+            if k in ("B", "T", "H", "D", "Ns"):
+                summary = re.sub(rf"\b{k}=\d+", f"{k}={v}", summary)
+        return dataclasses.replace(self, summary=summary, **kw)
+
+
+LAYER_WORKLOADS: Dict[str, LayerWorkload] = {
+    "layer": LayerWorkload("layer", 8, 2048, 4, 32, 16, "bf16", 5,
+                           summary="fused KLA layer forward, bf16 operators and values / fp32 state, "
+                                   "B=8 T=2048 H=4 D=32 Ns=16"),
+}
+
+LAYER_TOKEN_NAMES = ("k", "q", "v", "w")
+
+
+def generate_layer(w: LayerWorkload) -> Dict[str, np.ndarray]:
+    """Inputs of a layer workload as fp32 arrays: k, q [B, T, H, Ns] ~ N(0,
+    1/Ns); v [B, T, H, D] ~ N(0, 1); w (value precision) [B, T, H, D] =
+    softplus(N(0, 1)); a [H, D, Ns] = sigmoid(N(2, 1)) and p [H, D, Ns] =
+    softplus(N(-3, 1)) (the LM-layer families of a and p, time-invariant per
+    channel); prior lam0 = 1, eta0 = 0 [B, H, D, Ns].  k, q, v, w are rounded
+    to bf16 for bf16 workloads."""
+    children = np.random.SeedSequence([w.seed, 2]).spawn(6)
+    rngs = [np.random.Generator(np.random.PCG64(c)) for c in children]
+    B, T, H, D, Ns = w.B, w.T, w.H, w.D, w.Ns
+    rnd = (lambda x: round_to_bf16(x.astype(np.float32))) if w.dtype == "bf16" else \
+        (lambda x: x.astype(np.float32))
+    out = {
+        "k": rnd(rngs[0].standard_normal((B, T, H, Ns)) / np.sqrt(Ns)),
+        "q": rnd(rngs[1].standard_normal((B, T, H, Ns)) / np.sqrt(Ns)),
+        "v": rnd(rngs[2].standard_normal((B, T, H, D))),
+        "w": rnd(_softplus(rngs[3].standard_normal((B, T, H, D)))),
+        "a": _sigmoid(rngs[4].normal(2.0, 1.0, (H, D, Ns))).astype(np.float32),
+        "p": _softplus(rngs[5].normal(-3.0, 1.0, (H, D, Ns))).astype(np.float32),
+        "lam0": np.ones((B, H, D, Ns), dtype=np.float32),
+        "eta0": np.zeros((B, H, D, Ns), dtype=np.float32),
+    }
+    return out

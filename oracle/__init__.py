@@ -157,6 +157,60 @@ class Oracle:
             raise ValueError(f"kla_oracle_backward failed ({rc})")
         return out
 
+    def layer_forward(self, k, q, v, w, a, p, lam0, eta0, threads: int = 1):
+        """The KLA layer around the filter: evidence formed from the layer's
+        operators, the filter, and the readout.
+
+        Shapes: k, q [B, T, H, Ns] (observation and readout operators); v, w
+        [B, T, H, D] (values and their precision Lambda^v); a, p [H, D, Ns]
+        (time-invariant decay and process noise per state channel); lam0, eta0
+        [B, H, D, Ns] (prior).  State channel (h, d, n) is an independent
+        scalar filter observing value coordinate d through k_n:
+
+          phi = k_n^2 w_d,   b = k_n w_d v_d          (evidence precision and
+                                                       information, KLA review
+                                                       "Circularity Check")
+          y_d = sum_n q_n mu_{d,n},   s_d = sum_n q_n^2 var_{d,n}
+                                                      (readout of the posterior
+                                                       mean and of its variance
+                                                       under the diagonal posterior)
+
+        Returns fp64 ``y``, ``s`` [B, T, H, D] and the state after the last
+        token ``lam_T``, ``eta_T`` [B, H, D, Ns] (the prior when T = 0).
+        """
+        k, q, v, w = (_f64(x) for x in (k, q, v, w))
+        a, p = _f64(a), _f64(p)
+        if k.ndim != 4 or q.shape != k.shape or v.ndim != 4 or w.shape != v.shape:
+            raise ValueError("k, q must be [B, T, H, Ns] and v, w [B, T, H, D]")
+        B, T, H, Ns = k.shape
+        D = v.shape[3]
+        if v.shape[:3] != (B, T, H) or a.shape != (H, D, Ns) or p.shape != (H, D, Ns):
+            raise ValueError("v, w must be [B, T, H, D] and a, p [H, D, Ns]")
+        lam0 = _f64(np.broadcast_to(np.asarray(lam0, dtype=np.float64), (B, H, D, Ns)))
+        eta0 = _f64(np.broadcast_to(np.asarray(eta0, dtype=np.float64), (B, H, D, Ns)))
+        kk = k[:, :, :, None, :]                       # [B, T, H, 1, Ns]
+        ww = w[:, :, :, :, None]                       # [B, T, H, D, 1]
+        vv = v[:, :, :, :, None]
+        phi = kk * kk * ww                             # [B, T, H, D, Ns]
+        info = kk * ww * vv
+        shape5 = (B, T, H, D, Ns)
+        aa = np.broadcast_to(a, shape5)
+        pp = np.broadcast_to(p, shape5)
+        flat = lambda x: np.ascontiguousarray(x).reshape(B, T, H, D * Ns)
+        out = self.forward(flat(aa), flat(pp), flat(phi), flat(info),
+                           lam0.reshape(B, H, D * Ns), eta0.reshape(B, H, D * Ns), threads=threads)
+        mu = out["mu"].reshape(shape5)
+        var = out["var"].reshape(shape5)
+        qq = q[:, :, :, None, :]
+        y = np.sum(qq * mu, axis=4)
+        s_ = np.sum(qq * qq * var, axis=4)
+        if T > 0:
+            lam_T = out["lam"][:, T - 1].reshape(B, H, D, Ns)
+            eta_T = out["eta"][:, T - 1].reshape(B, H, D, Ns)
+        else:
+            lam_T, eta_T = lam0.copy(), eta0.copy()
+        return {"y": y, "s": s_, "lam_T": lam_T, "eta_T": eta_T}
+
 
 _DEFAULT: Oracle | None = None
 
@@ -180,3 +234,7 @@ def step(a, p, phi, b, lam_state, eta_state):
 def backward(a, p, phi, b, lam0, eta0, g_lam=None, g_eta=None, g_mu=None, g_var=None,
              threads: int = 1):
     return default().backward(a, p, phi, b, lam0, eta0, g_lam, g_eta, g_mu, g_var, threads=threads)
+
+
+def layer_forward(k, q, v, w, a, p, lam0, eta0, threads: int = 1):
+    return default().layer_forward(k, q, v, w, a, p, lam0, eta0, threads=threads)

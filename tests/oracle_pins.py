@@ -560,9 +560,104 @@ def pin_backward_closed_forms(orc):
         "p=0: eta does not depend on the precision path"
 
 
+# ------------------------------------------------------------ layer (fused)
+def random_rational_layer(seed, B=2, T=4, H=2, D=2, Ns=3):
+    rng = np.random.default_rng(seed)
+    def arr(shape, lo, hi, den, neg=False):
+        x = np.empty(shape, dtype=object)
+        for idx in np.ndindex(shape):
+            x[idx] = _random_fraction(rng, lo, hi, den) * (-1 if neg and rng.random() < 0.3 else 1)
+        return x
+    return {"k": arr((B, T, H, Ns), -5, 5, 4), "q": arr((B, T, H, Ns), -5, 5, 4),
+            "v": arr((B, T, H, D), -6, 6, 4), "w": arr((B, T, H, D), 1, 6, 4),
+            "a": arr((H, D, Ns), 1, 9, 8, neg=True), "p": arr((H, D, Ns), 0, 6, 8),
+            "lam0": arr((B, H, D, Ns), 1, 6, 4), "eta0": arr((B, H, D, Ns), -4, 4, 4)}
+
+
+def pin_layer_exact(orc, seeds=(31, 32)):
+    """The layer oracle == exact rationals done channel by channel with plain
+    loops: phi = k_n^2 w_d, b = k_n w_d v_d, the exact Moebius/affine filter,
+    y_d = sum_n q_n mu, s_d = sum_n q_n^2 var, final state = last posterior
+    (Ns = 3 and D = 2 so that a transposed or mis-broadcast axis shows)."""
+    for seed in seeds:
+        fr = random_rational_layer(seed)
+        B, T, H, Ns = fr["k"].shape
+        D = fr["v"].shape[3]
+        y = np.empty((B, T, H, D), dtype=object)
+        s_ = np.empty((B, T, H, D), dtype=object)
+        lam_T = np.empty((B, H, D, Ns), dtype=object)
+        eta_T = np.empty((B, H, D, Ns), dtype=object)
+        for bi in range(B):
+            for h in range(H):
+                for d in range(D):
+                    ysum = [Fr(0)] * T
+                    ssum = [Fr(0)] * T
+                    for n in range(Ns):
+                        ks = [fr["k"][bi, t, h, n] for t in range(T)]
+                        ws = [fr["w"][bi, t, h, d] for t in range(T)]
+                        vs = [fr["v"][bi, t, h, d] for t in range(T)]
+                        phi = [kk * kk * ww for kk, ww in zip(ks, ws)]
+                        info = [kk * ww * vv for kk, ww, vv in zip(ks, ws, vs)]
+                        lam, eta = exact_moebius_filter([fr["a"][h, d, n]] * T, [fr["p"][h, d, n]] * T, phi, info,
+                                                        fr["lam0"][bi, h, d, n], fr["eta0"][bi, h, d, n])
+                        for t in range(T):
+                            qq = fr["q"][bi, t, h, n]
+                            ysum[t] += qq * eta[t] / lam[t]
+                            ssum[t] += qq * qq / lam[t]
+                        lam_T[bi, h, d, n] = lam[-1]
+                        eta_T[bi, h, d, n] = eta[-1]
+                    for t in range(T):
+                        y[bi, t, h, d] = ysum[t]
+                        s_[bi, t, h, d] = ssum[t]
+        f64 = {kk: _to_f64(vv) for kk, vv in fr.items()}
+        got = orc.layer_forward(f64["k"], f64["q"], f64["v"], f64["w"], f64["a"], f64["p"],
+                                f64["lam0"], f64["eta0"])
+        _scaled_close(got["y"], _to_f64(y), 1e-12, f"layer y (seed {seed})")
+        _rel_close(got["s"], _to_f64(s_), 1e-12, f"layer s (seed {seed})")
+        _rel_close(got["lam_T"], _to_f64(lam_T), 1e-12, f"layer final lambda (seed {seed})")
+        _scaled_close(got["eta_T"].reshape(-1), _to_f64(eta_T).reshape(-1), 1e-12, f"layer final eta (seed {seed})",
+                      axis=None)
+
+
+def pin_layer_one_hot_readout(orc):
+    """A one-hot readout q = e_m returns the filter outputs of state channel m
+    (against the oracle's plain filter fed with phi = k_m^2 w, b = k_m w v), and
+    scaling q by c scales y by c and s by c^2."""
+    rng = np.random.default_rng(41)
+    B, T, H, D, Ns = 2, 30, 2, 3, 4
+    k = rng.standard_normal((B, T, H, Ns))
+    v = rng.standard_normal((B, T, H, D))
+    w = np.exp(rng.uniform(-1, 1, (B, T, H, D)))
+    a = rng.uniform(0.5, 1.0, (H, D, Ns))
+    p = np.exp(rng.uniform(np.log(1e-3), 0, (H, D, Ns)))
+    lam0 = np.exp(rng.uniform(-1, 1, (B, H, D, Ns)))
+    eta0 = rng.standard_normal((B, H, D, Ns))
+    for m in (0, Ns - 1):
+        q = np.zeros((B, T, H, Ns))
+        q[..., m] = 1.0
+        got = orc.layer_forward(k, q, v, w, a, p, lam0, eta0)
+        for h in range(H):
+            for d in range(D):
+                km = k[:, :, h, m]
+                ref = orc.forward(np.broadcast_to(a[h, d, m], (B, T)).reshape(B, T, 1, 1),
+                                  np.broadcast_to(p[h, d, m], (B, T)).reshape(B, T, 1, 1),
+                                  (km * km * w[:, :, h, d]).reshape(B, T, 1, 1),
+                                  (km * w[:, :, h, d] * v[:, :, h, d]).reshape(B, T, 1, 1),
+                                  lam0[:, h, d, m].reshape(B, 1, 1), eta0[:, h, d, m].reshape(B, 1, 1))
+                _scaled_close(got["y"][:, :, h, d], ref["mu"][:, :, 0, 0], 1e-13, f"one-hot y m={m}")
+                _rel_close(got["s"][:, :, h, d], ref["var"][:, :, 0, 0], 1e-13, f"one-hot s m={m}")
+    q = rng.standard_normal((B, T, H, Ns))
+    g1 = orc.layer_forward(k, q, v, w, a, p, lam0, eta0)
+    g3 = orc.layer_forward(k, -3.0 * q, v, w, a, p, lam0, eta0)
+    _scaled_close(g3["y"], -3.0 * g1["y"], 1e-14, "readout linear in q")
+    _rel_close(g3["s"], 9.0 * g1["s"], 1e-14, "variance readout quadratic in q")
+
+
+LAYER_PINS = [pin_layer_exact, pin_layer_one_hot_readout]
+
 BACKWARD_PINS = [pin_backward_exact_dual, pin_backward_autograd, pin_backward_finite_difference,
                  pin_backward_closed_forms]
 
 ALL_PINS = [pin_exact_rational, pin_exact_rational_step, pin_riccati, pin_precision_sum,
             pin_no_process_noise, pin_no_observation, pin_gate_derivative, pin_gate_product,
-            pin_invariants] + BACKWARD_PINS
+            pin_invariants] + BACKWARD_PINS + LAYER_PINS

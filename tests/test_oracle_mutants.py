@@ -71,3 +71,36 @@ def test_mutant_is_caught(name, tmp_path):
         except (AssertionError, ValueError, FloatingPointError, ZeroDivisionError) as e:
             failures.append((pin.__name__, str(e)[:80]))
     assert failures, f"no pin caught mutant {name!r}"
+
+
+# Mistakes planted in the layer function of the oracle package (Python source).
+LAYER_MUTANTS = {
+    "layer: phi = k w": ("phi = kk * kk * ww", "phi = kk * ww"),
+    "layer: information without the value precision": ("info = kk * ww * vv", "info = kk * vv"),
+    "layer: variance readout with q, not q^2": ("np.sum(qq * qq * var, axis=4)", "np.sum(qq * var, axis=4)"),
+    "layer: readout of eta": ('mu = out["mu"].reshape(shape5)', 'mu = out["eta"].reshape(shape5)'),
+    "layer: final state from the first token": ('lam_T = out["lam"][:, T - 1]', 'lam_T = out["lam"][:, 0]'),
+    "layer: k read out instead of q": ("qq = q[:, :, :, None, :]", "qq = k[:, :, :, None, :]"),
+    "layer: a and p swapped": ("self.forward(flat(aa), flat(pp),", "self.forward(flat(pp), flat(aa),"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(LAYER_MUTANTS))
+def test_layer_mutant_is_caught(name):
+    import importlib.util
+    old, new = LAYER_MUTANTS[name]
+    path = os.path.join(os.path.dirname(oracle.SOURCE), "__init__.py")
+    src = open(path).read()
+    assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+    spec = importlib.util.spec_from_loader("oracle_layer_mutant", loader=None, origin=path)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__file__ = path
+    exec(compile(src.replace(old, new), path, "exec"), mod.__dict__)
+    orc = mod.Oracle.load(oracle.build())
+    failures = []
+    for pin in pins.LAYER_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError, ZeroDivisionError) as e:
+            failures.append((pin.__name__, str(e)[:80]))
+    assert failures, f"no pin caught mutant {name!r}"
