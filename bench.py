@@ -6,8 +6,8 @@ cross-chunk carry, emit lambda / eta / mu / var) over the long-sequence
 workload (B=1, H=32, N=128, T=65536, fp32): 268.4 M token-channels per GPU,
 8.59 GB of algorithmic HBM traffic.  The same line also reports the recurrent
 decode step (B=256, H=32, N=128, fp32 resident state; 1024 tokens replayed
-from a CUDA graph) and the backward scan (kla_scan_backward) of the same
-workload.
+from a CUDA graph), the backward scan (kla_scan_backward) of the same
+workload, and the fused KLA layer (kla_layer_forward) on its own workload.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -337,6 +337,68 @@ def time_decode(kla, device, steps_tokens: int | None, replays: int):
             "note": "one kla_scan_step launch per token; the 8 MB fp32 state can stay L2-resident"}
 
 
+def time_layer(kla, device, steps: int, warmup: int):
+    """The fused KLA layer (kla_layer_forward) on the layer workload, and the
+    same computation unfused for comparison: phi, b, a, p formed with torch,
+    kla_scan_forward over the H x D x Ns channels, the readout with torch."""
+    import torch
+    w = wl.LAYER_WORKLOADS["layer"]
+    x = wl.generate_layer(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    d = {k: torch.from_numpy(x[k]).to(device).to(dt) for k in wl.LAYER_TOKEN_NAMES}
+    for k in ("a", "p", "lam0", "eta0"):
+        d[k] = torch.from_numpy(x[k]).to(device)
+    B, T, H, D, Ns = w.B, w.T, w.H, w.D, w.Ns
+    outs = [torch.empty((B, T, H, D), device=device), torch.empty((B, T, H, D), device=device),
+            torch.empty((B, H, D, Ns), device=device), torch.empty((B, H, D, Ns), device=device)]
+    ws = torch.empty(max(kla.layer_workspace_size(B, T, H, D, Ns, dt), 1), dtype=torch.uint8, device=device)
+    args = (d["k"], d["q"], d["v"], d["w"], d["a"], d["p"], d["lam0"], d["eta0"])
+
+    def fused():
+        kla.layer_forward(*args, out=outs, workspace=ws)
+
+    def unfused():
+        kk = d["k"].float()[:, :, :, None, :]
+        ww = d["w"].float()[:, :, :, :, None]
+        phi = (kk * kk * ww).reshape(B, T, H, D * Ns)
+        info = (kk * ww * d["v"].float()[:, :, :, :, None]).reshape(B, T, H, D * Ns)
+        aa = d["a"].expand(B, T, H, D, Ns).reshape(B, T, H, D * Ns).contiguous()
+        pp = d["p"].expand(B, T, H, D, Ns).reshape(B, T, H, D * Ns).contiguous()
+        lam, eta, mu, var = kla.scan_forward(aa, pp, phi, info, d["lam0"].reshape(B, H, D * Ns),
+                                             d["eta0"].reshape(B, H, D * Ns))
+        qq = d["q"].float()[:, :, :, None, :]
+        (qq * mu.reshape(B, T, H, D, Ns)).sum(-1)
+        (qq * qq * var.reshape(B, T, H, D, Ns)).sum(-1)
+
+    def timed(fn, n):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        if kla.get_error() != 0:
+            raise RuntimeError("device-side error in the layer warm-up")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for e0, e1 in ev:
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        if kla.get_error() != 0:
+            raise RuntimeError("device-side error in the timed layer region")
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    ms = timed(fused, steps)
+    ms_unfused = timed(unfused, max(3, steps // 10))
+    tc = w.token_channels
+    esz = 2 if w.dtype == "bf16" else 4
+    bytes_call = B * T * H * (2 * Ns * esz + 2 * D * esz + 2 * D * 4) + 4 * B * H * D * Ns * 4 + 2 * H * D * Ns * 4
+    return {"workload": f"{w.name}: {w.summary}", "ms_per_step": ms, "value": tc / (ms * 1e-3), "unit": UNIT,
+            "steps": steps, "kernel": "kla_layer_forward_kernel", "gpu_launches": steps,
+            "algorithmic_bytes_per_call": bytes_call, "gb_per_s": bytes_call / (ms * 1e-3) / 1e9,
+            "unfused_ms_per_step": ms_unfused, "speedup_vs_unfused": ms_unfused / ms,
+            "note": "ALU-bound: 0.9 B of HBM traffic per token-channel; the unfused path (torch forming phi, b, "
+                    "a, p and reading out, kla_scan_forward in between) moves about 40 B per token-channel"}
+
+
 def cpu_oracle_sample(w: wl.Workload, host_arrays, target_s: float = 10.0):
     """Time the fp64 oracle on a bounded sample of whole channels of the workload."""
     import oracle
@@ -413,6 +475,9 @@ def run_ours(args):
                                  (args.workload if not args.tokens else f"{args.workload}@T={args.tokens}")
                                  + ":backward")
     del fwd_outs
+    layer = None
+    if not args.no_layer:
+        layer = time_layer(kla, device, args.layer_steps, args.warmup)
 
     e2e = None
     if host is not None:
@@ -458,6 +523,7 @@ def run_ours(args):
         "e2e": e2e,
         "decode": decode,
         "backward": backward,
+        "layer": layer,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line))
@@ -517,6 +583,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-steps", type=int, default=50)
+    ap.add_argument("--no-layer", action="store_true")
+    ap.add_argument("--layer-steps", type=int, default=50)
     return ap.parse_args(argv)
 
 

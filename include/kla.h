@@ -320,6 +320,57 @@ kla_status_t kla_scan_backward_plan(int64_t B, int64_t T, int64_t H, int64_t N, 
 kla_status_t kla_debug_force_backward_kernel(int which);
 
 /*
+ * Device workspace that kla_layer_forward needs (run-boundary carries and
+ * flags, as for kla_scan_backward), written to *bytes; 0 when there is no
+ * token or no channel.  KLA_ERR_INVALID_ARG for negative sizes, a null
+ * `bytes`, Ns other than 8 or 16, or D not a multiple of 32 / Ns.
+ */
+kla_status_t kla_layer_forward_workspace_size(int64_t B, int64_t T, int64_t H, int64_t D, int64_t Ns,
+                                              kla_dtype_t in_dtype, size_t *bytes);
+
+/*
+ * The KLA layer's filter with its input formation and readout fused: for H
+ * heads of value dimension D and state expansion Ns, the H x D x Ns state
+ * channels (h, d, n) are independent scalar filters (the review's diagonal
+ * model) that observe value coordinate d through the observation operator
+ * k_n with the value precision w_d = Lambda^v_d:
+ *
+ *   phi_t = k_{t,n}^2 w_{t,d},  b_t = k_{t,n} w_{t,d} v_{t,d}   (the update adds
+ *          k^2 Lambda^v: review "Circularity Check", Theorem 1)
+ *   the filter above with the channel's time-invariant decay a and process
+ *          noise p (the review lists the OU decay as time-invariant; a and p
+ *          are taken already discretised)
+ *   y_{t,d} = sum_n q_{t,n} mu_{t,d,n},   s_{t,d} = sum_n q_{t,n}^2 var_{t,d,n}
+ *          (the readout operator q on the posterior mean, and the variance of
+ *          that readout under the diagonal posterior)
+ *
+ *   k, q          [B, T, H, Ns] observation / readout operators, in_dtype
+ *   v, w          [B, T, H, D] values and value precisions (w > 0), in_dtype
+ *   a, p          [H, D, Ns] fp32 per-channel decay and process noise (p >= 0)
+ *   lambda0, eta0 [B, H, D, Ns] fp32 prior
+ *   y             [B, T, H, D] fp32 readout (written)
+ *   s             [B, T, H, D] fp32 variance readout, or NULL
+ *   lambda_T, eta_T
+ *                 [B, H, D, Ns] fp32 state after the last token (for decoding
+ *                 on with kla_scan_step), or both NULL
+ *   workspace     at least kla_layer_forward_workspace_size(...) bytes,
+ *                 256-byte aligned (NULL when that is 0)
+ *
+ * Supported shapes: Ns = 8 or 16 (the state expansions the review lists),
+ * D a multiple of 32 / Ns; k, q, v, w 16-byte aligned.  Anything else returns
+ * KLA_ERR_INVALID_ARG before anything is enqueued (there is no fallback
+ * kernel).  T == 0 copies the prior into lambda_T / eta_T.  Outputs must not
+ * overlap inputs, the workspace or each other.  Results agree with
+ * kla_scan_forward on the formed phi, b followed by the readout, to rounding.
+ */
+kla_status_t kla_layer_forward(const void *k, const void *q, const void *v, const void *w,
+                               kla_dtype_t in_dtype, const float *a, const float *p,
+                               const float *lambda0, const float *eta0,
+                               float *y, float *s, float *lambda_T, float *eta_T,
+                               int64_t B, int64_t T, int64_t H, int64_t D, int64_t Ns,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Synchronise `stream`, then report the first failure since the previous
  * call on the current device: KLA_ERR_CUDA for a CUDA error (sticky or not),
  * KLA_ERR_TIMEOUT if a kernel's bounded wait ran out (the outputs that

@@ -58,6 +58,10 @@ SIGNATURES = {
     "kla_scan_backward_plan": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP,
                                               ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "kla_debug_force_backward_kernel": (ctypes.c_int, [ctypes.c_int]),
+    "kla_layer_forward_workspace_size": (ctypes.c_int, [_I64, _I64, _I64, _I64, _I64, ctypes.c_int,
+                                                        ctypes.POINTER(_SZ)]),
+    "kla_layer_forward": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                         _VP, _I64, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -420,3 +424,58 @@ def kalman_filter(a: torch.Tensor, p: torch.Tensor, phi: torch.Tensor, b: torch.
     """(lambda, eta, mu, var) of the filter, differentiable with respect to
     every input through the CUDA backward scan."""
     return KalmanFilterScan.apply(a, p, phi, b, lam0, eta0)
+
+
+# ------------------------------------------------------------ fused layer
+def layer_workspace_size(B: int, T: int, H: int, D: int, Ns: int, dtype: torch.dtype = torch.float32) -> int:
+    code = KLA_BF16 if dtype == torch.bfloat16 else KLA_F32
+    out = ctypes.c_size_t(0)
+    _check(lib().kla_layer_forward_workspace_size(B, T, H, D, Ns, code, ctypes.byref(out)),
+           "kla_layer_forward_workspace_size")
+    return int(out.value)
+
+
+def layer_forward(k: torch.Tensor, q: torch.Tensor, v: torch.Tensor, w: torch.Tensor,
+                  a: torch.Tensor, p: torch.Tensor, lam0: torch.Tensor, eta0: torch.Tensor, *,
+                  want_s: bool = True, want_state: bool = True,
+                  out: Optional[Sequence[Optional[torch.Tensor]]] = None,
+                  workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """The KLA layer's filter with evidence formation and readout fused
+    (kla_layer_forward): k, q [B, T, H, Ns]; v, w [B, T, H, D] (one dtype,
+    fp32 or bf16); a, p [H, D, Ns] fp32; lam0, eta0 [B, H, D, Ns] fp32.
+    Returns (y, s, lam_T, eta_T): y, s fp32 [B, T, H, D], the final state fp32
+    [B, H, D, Ns]; s / the state are None when not wanted."""
+    if k.dim() != 4 or q.shape != k.shape or v.dim() != 4 or w.shape != v.shape:
+        raise ValueError("k, q must be [B, T, H, Ns] and v, w [B, T, H, D]")
+    if not (k.dtype == q.dtype == v.dtype == w.dtype):
+        raise TypeError("k, q, v, w must share one dtype")
+    B, T, H, Ns = k.shape
+    D = v.shape[3]
+    if tuple(v.shape[:3]) != (B, T, H) or a.shape != (H, D, Ns) or p.shape != (H, D, Ns):
+        raise ValueError("v, w must be [B, T, H, D] and a, p [H, D, Ns]")
+    if lam0.shape != (B, H, D, Ns) or eta0.shape != (B, H, D, Ns):
+        raise ValueError("lam0 and eta0 must be [B, H, D, Ns]")
+    for t in (a, p, lam0, eta0):
+        if t.dtype != torch.float32:
+            raise TypeError("a, p, lam0, eta0 must be float32")
+    _require_cuda(k, q, v, w, a, p, lam0, eta0)
+    dev = k.device
+    if out is None:
+        outs = [torch.empty((B, T, H, D), dtype=torch.float32, device=dev),
+                torch.empty((B, T, H, D), dtype=torch.float32, device=dev) if want_s else None,
+                torch.empty((B, H, D, Ns), dtype=torch.float32, device=dev) if want_state else None,
+                torch.empty((B, H, D, Ns), dtype=torch.float32, device=dev) if want_state else None]
+    else:
+        outs = list(out)
+        _require_cuda(*outs)
+    if workspace is None:
+        n = layer_workspace_size(B, T, H, D, Ns, k.dtype)
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    with torch.cuda.device(dev):
+        st = lib().kla_layer_forward(
+            _ptr(k), _ptr(q), _ptr(v), _ptr(w), _dtype_code(k), _ptr(a), _ptr(p), _ptr(lam0), _ptr(eta0),
+            *[_ptr(o) for o in outs], B, T, H, D, Ns,
+            _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream_handle(stream))
+    _check(st, "kla_layer_forward")
+    return tuple(outs)

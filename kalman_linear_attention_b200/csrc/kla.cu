@@ -19,6 +19,7 @@
 #include "kla_backward.cuh"
 #include "kla_forward.cuh"
 #include "kla_forward_stream.cuh"
+#include "kla_layer.cuh"
 #include "kla_step.cuh"
 
 #define KLA_API extern "C" __attribute__((visibility("default")))
@@ -901,4 +902,145 @@ KLA_API kla_status_t kla_debug_force_backward_kernel(int which) {
     if (which < 0 || which > 2) return KLA_ERR_INVALID_ARG;
     g_force_bwd_kernel.store(which);
     return KLA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// The fused KLA layer: kla_layer_forward (kernel in kla_layer.cuh).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Chunk warps and ring stages of the layer kernel.  Its stages are small
+// (k and q of 32 tokens, v and w of 32 / Ns value coordinates: 4.9 KB for
+// fp32, Ns = 16) and the readout adds shuffles to every token, so it runs 11
+// chunk warps (12 in all: 168 registers) over a 16-stage ring.
+#ifndef KLA_LAYER_W
+#define KLA_LAYER_W 11
+#endif
+#ifndef KLA_LAYER_NS
+#define KLA_LAYER_NS 16
+#endif
+constexpr int kLayerL = 32;
+
+template <typename Tin, int NSX>
+cudaError_t launch_layer(const kla::LayerParams &prm, const kla::LayerMaps &maps, cudaStream_t stream) {
+    using Cfg = kla::LayerTile<Tin, NSX, kLayerL, KLA_LAYER_W, KLA_LAYER_NS>;
+    static_assert(Cfg::SMEM <= 227 * 1024, "layer kernel shared memory");
+    auto kernel = kla::kla_layer_forward_kernel<Tin, NSX, kLayerL, KLA_LAYER_W, KLA_LAYER_NS>;
+    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
+    kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    return cudaGetLastError();
+}
+
+// [B, T, H, Ns] tensor viewed as dims {Ns, H, T, B}, box {Ns, 1, 32, 1}.
+bool encode_layer_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz, int64_t B,
+                      int64_t T, int64_t H, int64_t Ns) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)Ns, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)(Ns * esz), (cuuint64_t)(H * Ns * esz),
+                                   (cuuint64_t)(T * H * Ns * esz)};
+    const cuuint32_t box[4] = {(cuuint32_t)Ns, 1u, (cuuint32_t)kLayerL, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tiles of 32 state channels: (32 / Ns) value coordinates x Ns.
+bool layer_shape_ok(int64_t D, int64_t Ns) { return (Ns == 8 || Ns == 16) && D % (32 / Ns) == 0; }
+
+}  // namespace
+
+KLA_API kla_status_t kla_layer_forward_workspace_size(int64_t B, int64_t T, int64_t H, int64_t D, int64_t Ns,
+                                                      kla_dtype_t in_dtype, size_t *bytes) {
+    if (!bytes || B < 0 || T < 0 || H < 0 || D < 0 || Ns < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    if (!layer_shape_ok(D, Ns)) return KLA_ERR_INVALID_ARG;
+    int64_t BH = 0, tiles = 0;
+    if (!mul_ok(B, H, &BH) || !mul_ok(BH, D / (32 / Ns), &tiles)) return KLA_ERR_INVALID_ARG;
+    if (tiles == 0 || T == 0) {
+        *bytes = 0;
+        return KLA_OK;
+    }
+    *bytes = stream_ws_layout(tiles, KLA_STREAM_MAX_PARTS).total;
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_layer_forward(const void *k, const void *q, const void *v, const void *w,
+                                       kla_dtype_t in_dtype, const float *a, const float *p,
+                                       const float *lambda0, const float *eta0, float *y, float *s,
+                                       float *lambda_T, float *eta_T, int64_t B, int64_t T, int64_t H,
+                                       int64_t D, int64_t Ns, void *workspace, size_t workspace_bytes,
+                                       void *stream) {
+    if (B < 0 || T < 0 || H < 0 || D < 0 || Ns < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    if (!layer_shape_ok(D, Ns)) return KLA_ERR_INVALID_ARG;
+    if ((lambda_T == nullptr) != (eta_T == nullptr)) return KLA_ERR_INVALID_ARG;
+    int64_t BT = 0, BTH = 0, kq_elems = 0, vw_elems = 0, HD = 0, chans = 0, BH = 0;
+    if (!mul_ok(B, T, &BT) || !mul_ok(BT, H, &BTH) || !mul_ok(BTH, Ns, &kq_elems) || !mul_ok(BTH, D, &vw_elems) ||
+        !mul_ok(H, D, &HD) || !mul_ok(B, H, &BH) || !mul_ok(BH, D * Ns, &chans))
+        return KLA_ERR_INVALID_ARG;
+    if (chans == 0) return KLA_OK;
+    const size_t esz = dtype_size(in_dtype);
+    if (!a || !p || !lambda0 || !eta0) return KLA_ERR_INVALID_ARG;
+    if (T > 0 && (!k || !q || !v || !w || !y)) return KLA_ERR_INVALID_ARG;
+    const void *aligned_ins[4] = {k, q, v, w};
+    for (int i = 0; i < 4; ++i)
+        if (aligned_ins[i] && !aligned16(aligned_ins[i])) return KLA_ERR_INVALID_ARG;
+    const Range outs[4] = {range_of(y, vw_elems * 4), range_of(s, vw_elems * 4), range_of(lambda_T, chans * 4),
+                           range_of(eta_T, chans * 4)};
+    const Range ins[9] = {range_of(k, kq_elems * (int64_t)esz), range_of(q, kq_elems * (int64_t)esz),
+                          range_of(v, vw_elems * (int64_t)esz), range_of(w, vw_elems * (int64_t)esz),
+                          range_of(a, HD * Ns * 4), range_of(p, HD * Ns * 4), range_of(lambda0, chans * 4),
+                          range_of(eta0, chans * 4), range_of(workspace, (int64_t)workspace_bytes)};
+    if (any_overlap(outs, 4, ins, 9)) return KLA_ERR_INVALID_ARG;
+    size_t need = 0;
+    if (kla_layer_forward_workspace_size(B, T, H, D, Ns, in_dtype, &need) != KLA_OK) return KLA_ERR_INVALID_ARG;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KLA_ERR_WORKSPACE_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KLA_ERR_MISALIGNED;
+    if (T > INT32_MAX - 64 || H > INT32_MAX || D > INT32_MAX || B > INT32_MAX) return KLA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // no tokens: the final state is the prior
+        if (lambda_T) {
+            if (cudaMemcpyAsync(lambda_T, lambda0, (size_t)chans * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+                cudaMemcpyAsync(eta_T, eta0, (size_t)chans * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+                return KLA_ERR_CUDA;
+        }
+        return KLA_OK;
+    }
+    const CUtensorMapDataType tdt =
+        in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    kla::LayerMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!encode_layer_map(&maps.k, k, tdt, esz, B, T, H, Ns) || !encode_layer_map(&maps.q, q, tdt, esz, B, T, H, Ns))
+        return KLA_ERR_CUDA;
+    kla::LayerParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.v = v; prm.w = w; prm.a = a; prm.p = p; prm.lam0 = lambda0; prm.eta0 = eta0;
+    prm.y = y; prm.s = s; prm.lam_T = lambda_T; prm.eta_T = eta_T;
+    prm.T = T; prm.H = (int)H; prm.D = (int)D;
+    prm.dtiles = (int)(D / (32 / Ns));
+    prm.ntiles = BH * prm.dtiles;
+    prm.nchunks = (int)((T + kLayerL - 1) / kLayerL);
+    prm.wait_ns = g_wait_ns.load();
+    prm.parts = stream_parts(prm.ntiles, prm.nchunks);
+    prm.chunks_per_part = (prm.nchunks + prm.parts - 1) / prm.parts;
+    prm.nunits = prm.ntiles * prm.parts;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    prm.ticket = reinterpret_cast<unsigned *>(ws);
+    if (prm.parts > 1) {
+        const StreamWs sw = stream_ws_layout(prm.ntiles, prm.parts);
+        prm.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
+        prm.part_state = reinterpret_cast<float *>(ws + sw.state_off);
+        if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
+    }
+    cudaError_t e;
+    if (in_dtype == KLA_F32)
+        e = Ns == 8 ? launch_layer<float, 8>(prm, maps, st) : launch_layer<float, 16>(prm, maps, st);
+    else
+        e = Ns == 8 ? launch_layer<__nv_bfloat16, 8>(prm, maps, st) : launch_layer<__nv_bfloat16, 16>(prm, maps, st);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }

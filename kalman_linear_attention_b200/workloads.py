@@ -310,3 +310,11 @@ def generate_layer(w: LayerWorkload) -> Dict[str, np.ndarray]:
         "eta0": np.zeros((B, H, D, Ns), dtype=np.float32),
     }
     return out
+
+
+def random_layer_prior(w: LayerWorkload, seed: int = 778) -> Dict[str, np.ndarray]:
+    """A non-trivial layer prior: lam0 ~ logU(0.1, 10), eta0 ~ N(0, 1), fp32 [B, H, D, Ns]."""
+    rng = np.random.default_rng([w.seed, seed])
+    shape = (w.B, w.H, w.D, w.Ns)
+    return {"lam0": _log_uniform(rng, 0.1, 10.0, int(np.prod(shape))).astype(np.float32).reshape(shape),
+            "eta0": rng.standard_normal(shape).astype(np.float32)}
