@@ -160,3 +160,33 @@ def test_backward_host_argument_errors(lib):
     assert lib.kla_scan_backward_plan(1, 64, 32, 128, 0, P + 4, P, ctypes.byref(k), ctypes.byref(n)) == 0
     assert k.value == 1                                       # unaligned input
     assert lib.kla_debug_force_backward_kernel(3) == 1
+
+
+def test_layer_host_argument_errors(lib):
+    """kla_layer_forward: shape, pointer, alignment and overlap checks answer on
+    the host."""
+    f = lib.kla_layer_forward
+    P = 1 << 20  # fake, never dereferenced
+    names = ["k", "q", "v", "w", "dt", "a", "p", "lam0", "eta0", "y", "s", "lamT", "etaT",
+             "B", "T", "H", "D", "Ns", "ws", "wsb", "stream"]
+    base = dict(k=P, q=2 * P, v=3 * P, w=4 * P, dt=0, a=5 * P, p=6 * P, lam0=7 * P, eta0=8 * P, y=9 * P,
+                s=10 * P, lamT=11 * P, etaT=12 * P, B=1, T=64, H=2, D=4, Ns=16, ws=16 * P, wsb=1 << 20, stream=None)
+    args = lambda **kw: [kw.get(n, base[n]) for n in names]
+    assert f(*args(Ns=4)) == 1                  # unsupported state expansion
+    assert f(*args(Ns=32)) == 1
+    assert f(*args(D=3)) == 1                   # D not a multiple of 32 / Ns
+    assert f(*args(dt=5)) == 2
+    assert f(*args(k=None)) == 1
+    assert f(*args(a=None)) == 1
+    assert f(*args(lamT=None)) == 1             # final state: both or neither
+    assert f(*args(k=P + 4)) == 1               # k not 16-byte aligned
+    assert f(*args(y=P)) == 1                   # y overlaps k
+    assert f(*args(s=9 * P)) == 1               # s overlaps y
+    assert f(*args(wsb=16)) == 3
+    assert f(*args(ws=16 * P + 8)) == 6
+    assert f(*args(B=0)) == 0                   # no channels: nothing enqueued
+    out = ctypes.c_size_t(7)
+    assert lib.kla_layer_forward_workspace_size(8, 2048, 4, 32, 16, 1, ctypes.byref(out)) == 0
+    assert out.value > 0
+    assert lib.kla_layer_forward_workspace_size(8, 0, 4, 32, 16, 1, ctypes.byref(out)) == 0 and out.value == 0
+    assert lib.kla_layer_forward_workspace_size(8, 16, 4, 30, 8, 1, ctypes.byref(out)) == 1
