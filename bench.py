@@ -388,6 +388,41 @@ def time_layer(kla, device, steps: int, warmup: int):
 
     ms = timed(fused, steps)
     ms_unfused = timed(unfused, max(3, steps // 10))
+
+    # decode: kla_layer_step tokens from a CUDA graph (B = 256 sequences)
+    Bd, Td = 256, 256
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 29)
+    dk = (torch.randn((Td, Bd, H, Ns), generator=gen, device=device) / Ns ** 0.5).to(dt)
+    dq = (torch.randn((Td, Bd, H, Ns), generator=gen, device=device) / Ns ** 0.5).to(dt)
+    dv = torch.randn((Td, Bd, H, D), generator=gen, device=device).to(dt)
+    dw = torch.nn.functional.softplus(torch.randn((Td, Bd, H, D), generator=gen, device=device)).to(dt)
+    lam = torch.ones((Bd, H, D, Ns), device=device)
+    eta = torch.zeros((Bd, H, D, Ns), device=device)
+    yd = torch.empty((Bd, H, D), device=device)
+    sd = torch.empty((Bd, H, D), device=device)
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        for t in range(3):
+            kla.layer_step(dk[t], dq[t], dv[t], dw[t], d["a"], d["p"], lam, eta, y=yd, s=sd, stream=st)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=st):
+        for t in range(Td):
+            kla.layer_step(dk[t], dq[t], dv[t], dw[t], d["a"], d["p"], lam, eta, y=yd, s=sd, stream=st)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(4):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error in the layer decode")
+    us_token = e0.elapsed_time(e1) * 1e3 / (4 * Td)
+    del graph
     tc = w.token_channels
     esz = 2 if w.dtype == "bf16" else 4
     bytes_call = B * T * H * (2 * Ns * esz + 2 * D * esz + 2 * D * 4) + 4 * B * H * D * Ns * 4 + 2 * H * D * Ns * 4
@@ -395,6 +430,9 @@ def time_layer(kla, device, steps: int, warmup: int):
             "steps": steps, "kernel": "kla_layer_forward_kernel", "gpu_launches": steps,
             "algorithmic_bytes_per_call": bytes_call, "gb_per_s": bytes_call / (ms * 1e-3) / 1e9,
             "unfused_ms_per_step": ms_unfused, "speedup_vs_unfused": ms_unfused / ms,
+            "decode": {"us_per_token": us_token, "batch": Bd,
+                       "token_channels_per_s": Bd * H * D * Ns / (us_token * 1e-6),
+                       "how": f"kla_layer_step, {Td} tokens captured in a CUDA graph, 4 replays"},
             "note": "ALU-bound: 0.9 B of HBM traffic per token-channel; the unfused path (torch forming phi, b, "
                     "a, p and reading out, kla_scan_forward in between) moves about 40 B per token-channel"}
 

@@ -48,7 +48,9 @@
  *   Any real a_t is allowed (only a_t^2 enters the precision; the sign of a_t
  *   enters the gate).
  * - Arithmetic: inputs are fp32 or bf16 (converted exactly to fp32 on load);
- *   state and outputs are fp32 with IEEE division; no fast-math.
+ *   state, arithmetic and outputs are fp32 (the gradients of an input are
+ *   written in that input's dtype); reciprocals use the hardware instruction
+ *   (PTX rcp.approx.ftz.f32, within 1 ulp); nothing else is approximated.
  * - Outputs must not overlap inputs or each other.
  */
 #ifndef KLA_H
@@ -369,6 +371,27 @@ kla_status_t kla_layer_forward(const void *k, const void *q, const void *v, cons
                                float *y, float *s, float *lambda_T, float *eta_T,
                                int64_t B, int64_t T, int64_t H, int64_t D, int64_t Ns,
                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode token of the fused layer, from the resident state: the
+ * recurrent counterpart of kla_layer_forward (continue from its lambda_T /
+ * eta_T).  Same channels, evidence, filter and readout, for one token.
+ *
+ *   k, q          [B, H, Ns] this token's operators, in_dtype
+ *   v, w          [B, H, D] this token's values and value precisions, in_dtype
+ *   a, p          [H, D, Ns] fp32
+ *   lambda_state, eta_state
+ *                 [B, H, D, Ns] fp32 state, read and overwritten in place
+ *   y             [B, H, D] fp32 readout of this token (written)
+ *   s             [B, H, D] fp32 variance readout, or NULL
+ *
+ * Ns = 8 or 16 and D a multiple of 32 / Ns (KLA_ERR_INVALID_ARG otherwise);
+ * any alignment.  B*H*D == 0 is valid (nothing is enqueued).  Outputs must
+ * not overlap the inputs or each other.
+ */
+kla_status_t kla_layer_step(const void *k, const void *q, const void *v, const void *w, kla_dtype_t in_dtype,
+                            const float *a, const float *p, float *lambda_state, float *eta_state,
+                            float *y, float *s, int64_t B, int64_t H, int64_t D, int64_t Ns, void *stream);
 
 /*
  * Synchronise `stream`, then report the first failure since the previous

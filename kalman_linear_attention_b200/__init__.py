@@ -12,7 +12,7 @@ _API_NAMES = {
     "debug_force_forward_kernel", "forward_plan", "host_workspace_size",
     "KlaError", "lib", "load_library", "scan_forward_static",
     "scan_backward", "backward_workspace_size", "backward_plan", "debug_force_backward_kernel",
-    "KalmanFilterScan", "kalman_filter", "layer_forward", "layer_workspace_size",
+    "KalmanFilterScan", "kalman_filter", "layer_forward", "layer_workspace_size", "layer_step",
 }
 
 

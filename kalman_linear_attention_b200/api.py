@@ -62,6 +62,8 @@ SIGNATURES = {
                                                         ctypes.POINTER(_SZ)]),
     "kla_layer_forward": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                          _VP, _I64, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
+    "kla_layer_step": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP,
+                                      _I64, _I64, _I64, _I64, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -479,3 +481,31 @@ def layer_forward(k: torch.Tensor, q: torch.Tensor, v: torch.Tensor, w: torch.Te
             _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream_handle(stream))
     _check(st, "kla_layer_forward")
     return tuple(outs)
+
+
+def layer_step(k: torch.Tensor, q: torch.Tensor, v: torch.Tensor, w: torch.Tensor,
+               a: torch.Tensor, p: torch.Tensor, lam_state: torch.Tensor, eta_state: torch.Tensor, *,
+               y: Optional[torch.Tensor] = None, s: Optional[torch.Tensor] = None, want_s: bool = True,
+               stream: Optional[torch.cuda.Stream] = None):
+    """One decode token of the fused layer (kla_layer_step): k, q [B, H, Ns];
+    v, w [B, H, D]; a, p [H, D, Ns]; the state [B, H, D, Ns] is updated in
+    place.  Returns (y, s), fp32 [B, H, D] (s None when not wanted)."""
+    if k.dim() != 3 or q.shape != k.shape or v.dim() != 3 or w.shape != v.shape:
+        raise ValueError("k, q must be [B, H, Ns] and v, w [B, H, D]")
+    if not (k.dtype == q.dtype == v.dtype == w.dtype):
+        raise TypeError("k, q, v, w must share one dtype")
+    B, H, Ns = k.shape
+    D = v.shape[2]
+    if tuple(v.shape[:2]) != (B, H) or lam_state.shape != (B, H, D, Ns) or eta_state.shape != (B, H, D, Ns):
+        raise ValueError("v, w must be [B, H, D] and the state [B, H, D, Ns]")
+    _require_cuda(k, q, v, w, a, p, lam_state, eta_state, y, s)
+    if y is None:
+        y = torch.empty((B, H, D), dtype=torch.float32, device=k.device)
+    if s is None and want_s:
+        s = torch.empty((B, H, D), dtype=torch.float32, device=k.device)
+    with torch.cuda.device(k.device):
+        st = lib().kla_layer_step(_ptr(k), _ptr(q), _ptr(v), _ptr(w), _dtype_code(k), _ptr(a), _ptr(p),
+                                  _ptr(lam_state), _ptr(eta_state), _ptr(y), _ptr(s), B, H, D, Ns,
+                                  _stream_handle(stream))
+    _check(st, "kla_layer_step")
+    return y, s

@@ -1044,3 +1044,50 @@ KLA_API kla_status_t kla_layer_forward(const void *k, const void *q, const void 
         e = Ns == 8 ? launch_layer<__nv_bfloat16, 8>(prm, maps, st) : launch_layer<__nv_bfloat16, 16>(prm, maps, st);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
+
+KLA_API kla_status_t kla_layer_step(const void *k, const void *q, const void *v, const void *w,
+                                    kla_dtype_t in_dtype, const float *a, const float *p, float *lambda_state,
+                                    float *eta_state, float *y, float *s, int64_t B, int64_t H, int64_t D,
+                                    int64_t Ns, void *stream) {
+    if (B < 0 || H < 0 || D < 0 || Ns < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    if (!layer_shape_ok(D, Ns)) return KLA_ERR_INVALID_ARG;
+    int64_t BH = 0, DN = 0, C = 0, HDN = 0, BHD = 0;
+    if (!mul_ok(B, H, &BH) || !mul_ok(D, Ns, &DN) || !mul_ok(BH, DN, &C) || !mul_ok(H, DN, &HDN) ||
+        !mul_ok(BH, D, &BHD))
+        return KLA_ERR_INVALID_ARG;
+    if (C == 0) return KLA_OK;
+    if (!k || !q || !v || !w || !a || !p || !lambda_state || !eta_state || !y) return KLA_ERR_INVALID_ARG;
+    if (DN > INT32_MAX) return KLA_ERR_INVALID_ARG;
+    const int64_t esz = (int64_t)dtype_size(in_dtype);
+    const Range outs[4] = {range_of(lambda_state, C * 4), range_of(eta_state, C * 4), range_of(y, BHD * 4),
+                           range_of(s, BHD * 4)};
+    const Range ins[6] = {range_of(k, BH * Ns * esz), range_of(q, BH * Ns * esz), range_of(v, BHD * esz),
+                          range_of(w, BHD * esz), range_of(a, HDN * 4), range_of(p, HDN * 4)};
+    if (any_overlap(outs, 4, ins, 6)) return KLA_ERR_INVALID_ARG;
+    kla::LayerStepParams prm;
+    prm.k = k; prm.q = q; prm.v = v; prm.w = w; prm.a = a; prm.p = p;
+    prm.lam = lambda_state; prm.eta = eta_state; prm.y = y; prm.s = s;
+    prm.C = C; prm.HDN = HDN; prm.DN = (int)DN;
+    const int threads = 256;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((C + threads - 1) / threads, 148 * 16));
+    // programmatic dependent launch, as for kla_scan_step
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (in_dtype == KLA_F32)
+        e = Ns == 8 ? cudaLaunchKernelEx(&cfg, kla::kla_layer_step_kernel<float, 8>, prm)
+                    : cudaLaunchKernelEx(&cfg, kla::kla_layer_step_kernel<float, 16>, prm);
+    else
+        e = Ns == 8 ? cudaLaunchKernelEx(&cfg, kla::kla_layer_step_kernel<__nv_bfloat16, 8>, prm)
+                    : cudaLaunchKernelEx(&cfg, kla::kla_layer_step_kernel<__nv_bfloat16, 16>, prm);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}

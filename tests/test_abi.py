@@ -190,3 +190,19 @@ def test_layer_host_argument_errors(lib):
     assert out.value > 0
     assert lib.kla_layer_forward_workspace_size(8, 0, 4, 32, 16, 1, ctypes.byref(out)) == 0 and out.value == 0
     assert lib.kla_layer_forward_workspace_size(8, 16, 4, 30, 8, 1, ctypes.byref(out)) == 1
+
+
+def test_layer_step_host_argument_errors(lib):
+    f = lib.kla_layer_step
+    P = 1 << 20
+    names = ["k", "q", "v", "w", "dt", "a", "p", "lam", "eta", "y", "s", "B", "H", "D", "Ns", "stream"]
+    base = dict(k=P, q=2 * P, v=3 * P, w=4 * P, dt=0, a=5 * P, p=6 * P, lam=7 * P, eta=8 * P, y=9 * P, s=None,
+                B=2, H=2, D=4, Ns=16, stream=None)
+    args = lambda **kw: [kw.get(n, base[n]) for n in names]
+    assert f(*args(Ns=4)) == 1
+    assert f(*args(D=5)) == 1
+    assert f(*args(dt=3)) == 2
+    assert f(*args(lam=None)) == 1
+    assert f(*args(y=P)) == 1          # y overlaps k
+    assert f(*args(eta=7 * P)) == 1    # state halves overlap
+    assert f(*args(B=0)) == 0

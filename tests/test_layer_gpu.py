@@ -190,3 +190,40 @@ def test_layer_full_size_sampled():
             worst[k] = max(worst.get(k, 0.0), v)
     print("layer full-size sampled max errors", worst)
     assert max(worst.values()) <= parity.RTOL[w.dtype], worst
+
+
+@pytest.mark.parametrize("dtype,Ns", [("f32", 16), ("bf16", 8)])
+def test_layer_prefill_then_decode(dtype, Ns):
+    """kla_layer_forward over the first tokens, then kla_layer_step token by
+    token from its final state: every decoded readout and the final state
+    against the oracle over the whole sequence, and the decoded readouts
+    against the fused kernel's own rows over the same tokens."""
+    import dataclasses
+    kla = _kla()
+    w = dataclasses.replace(wl.LAYER_WORKLOADS["layer"].with_shape(B=2, T=80, H=2, D=4, Ns=Ns), dtype=dtype)
+    x = wl.generate_layer(w)
+    x.update(wl.random_layer_prior(w))
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    d = to_dev(x, dt)
+    ref = oracle.layer_forward(x["k"], x["q"], x["v"], x["w"], x["a"], x["p"], x["lam0"], x["eta0"])
+    full = kla.layer_forward(d["k"], d["q"], d["v"], d["w"], d["a"], d["p"], d["lam0"], d["eta0"])
+    T1 = 50
+    pre = kla.layer_forward(d["k"][:, :T1].contiguous(), d["q"][:, :T1].contiguous(), d["v"][:, :T1].contiguous(),
+                            d["w"][:, :T1].contiguous(), d["a"], d["p"], d["lam0"], d["eta0"])
+    lam, eta = pre[2].clone(), pre[3].clone()
+    ys, ss = [], []
+    for t in range(T1, w.T):
+        y, s = kla.layer_step(d["k"][:, t].contiguous(), d["q"][:, t].contiguous(), d["v"][:, t].contiguous(),
+                              d["w"][:, t].contiguous(), d["a"], d["p"], lam, eta)
+        ys.append(y.clone())
+        ss.append(s.clone())
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {"y": torch.stack(ys, 1).double().cpu().numpy(), "s": torch.stack(ss, 1).double().cpu().numpy(),
+           "lam_T": lam.double().cpu().numpy(), "eta_T": eta.double().cpu().numpy()}
+    tail = {"y": ref["y"][:, T1:], "s": ref["s"][:, T1:], "lam_T": ref["lam_T"], "eta_T": ref["eta_T"]}
+    errs = layer_errors(got, tail)
+    assert max(errs.values()) <= 1e-5, errs
+    own = {"y": full[0][:, T1:].double().cpu().numpy(), "s": full[1][:, T1:].double().cpu().numpy(),
+           "lam_T": full[2].double().cpu().numpy(), "eta_T": full[3].double().cpu().numpy()}
+    assert max(layer_errors(got, own).values()) <= 2e-6
