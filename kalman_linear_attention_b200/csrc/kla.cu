@@ -1068,12 +1068,14 @@ KLA_API kla_status_t kla_layer_step(const void *k, const void *q, const void *v,
     kla::LayerStepParams prm;
     prm.k = k; prm.q = q; prm.v = v; prm.w = w; prm.a = a; prm.p = p;
     prm.lam = lambda_state; prm.eta = eta_state; prm.y = y; prm.s = s;
-    prm.C = C; prm.HDN = HDN; prm.DN = (int)DN;
+    prm.BH = BH; prm.H = (int)H; prm.D = (int)D; prm.DN = (int)DN;
+    if (HDN > INT32_MAX || BH > INT32_MAX) return KLA_ERR_INVALID_ARG;
     const int threads = 256;
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((C + threads - 1) / threads, 148 * 16));
+    const int64_t bx = (DN + threads - 1) / threads;
+    const int64_t by = std::max<int64_t>(1, std::min<int64_t>(BH, std::max<int64_t>(1, 148 * 16 / bx)));
     // programmatic dependent launch, as for kla_scan_step
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.gridDim = dim3((unsigned)bx, (unsigned)std::min<int64_t>(by, 65535));
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = static_cast<cudaStream_t>(stream);

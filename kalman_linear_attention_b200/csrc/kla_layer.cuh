@@ -367,44 +367,46 @@ kla_layer_forward_kernel(const LayerParams prm, const __grid_constant__ LayerMap
 
 // ---------------------------------------------------------------------------
 // One decode token of the layer: the recurrent counterpart of the kernel
-// above (as kla_step_*_kernel is of the scan).  One thread per state channel
-// c = ((b H + h) D + d) Ns + n; a warp holds 32 / Ns whole value coordinates
-// (D Ns is a multiple of 32), so the readout reduces over lanes as above.
+// above (as kla_step_*_kernel is of the scan).  Grid y runs over the B H
+// (sequence, head) rows, grid x over the D Ns state channels of a row, one
+// thread per channel c = d Ns + n; a warp holds 32 / Ns whole value
+// coordinates (D Ns is a multiple of 32), so the readout reduces over lanes
+// as above.  No index division in the loop.
 struct LayerStepParams {
     const void *k, *q;             // [B, H, Ns] this token's operators
     const void *v, *w;             // [B, H, D] this token's values and precisions
     const float *a, *p;            // [H, D, Ns]
     float *lam, *eta;              // [B, H, D, Ns] state, in place
     float *y, *s;                  // [B, H, D]; s may be null
-    int64_t C;                     // B H D Ns
-    int64_t HDN;                   // H D Ns
-    int DN;                        // D Ns
+    int64_t BH;                    // B H rows
+    int H, D, DN;                  // DN = D Ns
 };
 
 template <typename Tin, int NSX>
 __global__ void __launch_bounds__(256) kla_layer_step_kernel(const LayerStepParams prm) {
     grid_dependency_wait();
     allow_dependent_launch();
-    const int lane = threadIdx.x & 31;
-    const int n = lane % NSX;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;    // channel within the row
+    if (c >= prm.DN) return;                                // whole warps (DN is a multiple of 32)
+    const int n = c % NSX;
+    const int d = c / NSX;
     const Tin *kg = static_cast<const Tin *>(prm.k);
     const Tin *qg = static_cast<const Tin *>(prm.q);
     const Tin *vg = static_cast<const Tin *>(prm.v);
     const Tin *wg = static_cast<const Tin *>(prm.w);
-    // whole warps only (C is a multiple of 32), so every shuffle has its partners
-    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < prm.C;
-         c += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t vd = c / NSX;                     // (b H + h) D + d
-        const int64_t bh = c / prm.DN;                  // b H + h
+    for (int64_t bh = blockIdx.y; bh < prm.BH; bh += gridDim.y) {
+        const int h = (int)((unsigned)bh % (unsigned)prm.H);   // B H < 2^31
+        const int64_t row = bh * prm.DN + c;                 // [B, H, D, Ns] index
+        const int64_t vd = bh * prm.D + d;                   // [B, H, D] index
         const float kk = to_f32(kg[bh * NSX + n]);
         const float qq = to_f32(qg[bh * NSX + n]);
         const float ww = to_f32(wg[vd]);
         const float vv = to_f32(vg[vd]);
-        const int64_t pc = c % prm.HDN;
-        float lam = prm.lam[c], eta = prm.eta[c];
+        const int pc = h * prm.DN + c;
+        float lam = prm.lam[row], eta = prm.eta[row];
         const TokenOut o = filter_token(lam, eta, prm.a[pc], prm.p[pc], (kk * kk) * ww, (kk * ww) * vv);
-        prm.lam[c] = lam;
-        prm.eta[c] = eta;
+        prm.lam[row] = lam;
+        prm.eta[row] = eta;
         float ym = qq * o.mu;
         float sv2 = (qq * qq) * o.var;
 #pragma unroll
