@@ -318,3 +318,40 @@ def random_layer_prior(w: LayerWorkload, seed: int = 778) -> Dict[str, np.ndarra
     shape = (w.B, w.H, w.D, w.Ns)
     return {"lam0": _log_uniform(rng, 0.1, 10.0, int(np.prod(shape))).astype(np.float32).reshape(shape),
             "eta0": rng.standard_normal(shape).astype(np.float32)}
+
+
+SPECIAL_CASES = ["no_process_noise", "no_observation", "precision_sum", "negative_decay", "mixed_zeros"]
+
+
+def special_inputs(kind: str, B: int = 2, T: int = 400, H: int = 2, N: int = 48, seed: int = 77
+                   ) -> Dict[str, np.ndarray]:
+    """Degenerate and special cases of the method, seeded, fp32: p = 0 with
+    a near +-1 (the affine Moebius case), phi = b = 0 (no observation), a = 1
+    and p = 0 (precision sum), a of either sign, and a mix of zero noise and
+    missing observations; a non-trivial prior."""
+    rng = np.random.default_rng(seed)
+    sh = (B, T, H, N)
+    a = rng.uniform(0.5, 1.0, sh)
+    p = np.exp(rng.uniform(np.log(1e-3), 0.0, sh))
+    phi = np.exp(rng.uniform(np.log(1e-2), np.log(10.0), sh))
+    b = rng.standard_normal(sh)
+    if kind == "no_process_noise":      # p = 0: the affine Moebius case
+        p[:] = 0.0
+        a = rng.uniform(0.98, 1.02, sh) * np.where(rng.random(sh) < 0.3, -1.0, 1.0)
+    elif kind == "no_observation":      # phi = 0, b = 0: every update leaves the prior
+        phi[:] = 0.0
+        b[:] = 0.0
+    elif kind == "precision_sum":       # a = 1, p = 0: lambda is a running sum of phi
+        a[:] = 1.0
+        p[:] = 0.0
+    elif kind == "negative_decay":      # the gate follows the sign of a
+        a *= np.where(rng.random(sh) < 0.5, -1.0, 1.0)
+    elif kind == "mixed_zeros":         # some tokens without noise, some without evidence
+        p[rng.random(sh) < 0.3] = 0.0
+        z = rng.random(sh) < 0.3
+        phi[z] = 0.0
+        b[z] = 0.0
+    x = {k: v.astype(np.float32) for k, v in (("a", a), ("p", p), ("phi", phi), ("b", b))}
+    x["lam0"] = rng.uniform(0.5, 2.0, (B, H, N)).astype(np.float32)
+    x["eta0"] = rng.standard_normal((B, H, N)).astype(np.float32)
+    return x

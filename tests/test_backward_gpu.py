@@ -255,3 +255,26 @@ def test_backward_full_size_sampled(name, count):
     w, errs = _sampled_full_size(name, count)
     print(name, "backward max scaled errors", errs)
     assert max(errs.values()) <= parity.RTOL[w.dtype], errs
+
+
+@pytest.mark.parametrize("kind", wl.SPECIAL_CASES)
+def test_backward_special_cases(kind, kernel):
+    """Gradients in the degenerate cases of the method: no process noise
+    (a near +-1), no observation (phi = b = 0), the precision sum (a = 1,
+    p = 0), negative decay and mixed zeros, against the oracle, with all four
+    output gradients present."""
+    kla = _kla()
+    x = wl.special_inputs(kind, T=300)
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=300, H=2, N=48)
+    go = wl.generate_output_grads(w)
+    d = {k: torch.from_numpy(v).to(DEV) for k, v in x.items()}
+    lam, eta, _, _ = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"],
+                                      want_mu=False, want_var=False)
+    g = [torch.from_numpy(go[k]).to(DEV) for k in wl.GRAD_NAMES]
+    out = kla.scan_backward(d["a"], d["p"], d["lam0"], d["eta0"], lam, eta, *g)
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(GRADS + ("lam0", "eta0"), out)}
+    ref = oracle.backward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"],
+                          *(go[k] for k in wl.GRAD_NAMES), threads=8)
+    assert_grad_parity(got, ref, parity.RTOL["f32"], what=kind)

@@ -234,37 +234,8 @@ def test_plan_matches_workloads():
         del z
 
 
-def _special_inputs(kind, B=2, T=400, H=2, N=48, seed=77):
-    """Degenerate and special cases of the method, seeded."""
-    rng = np.random.default_rng(seed)
-    sh = (B, T, H, N)
-    a = rng.uniform(0.5, 1.0, sh)
-    p = np.exp(rng.uniform(np.log(1e-3), 0.0, sh))
-    phi = np.exp(rng.uniform(np.log(1e-2), np.log(10.0), sh))
-    b = rng.standard_normal(sh)
-    if kind == "no_process_noise":      # p = 0: the affine Moebius case
-        p[:] = 0.0
-        a = rng.uniform(0.98, 1.02, sh) * np.where(rng.random(sh) < 0.3, -1.0, 1.0)
-    elif kind == "no_observation":      # phi = 0, b = 0: every update leaves the prior
-        phi[:] = 0.0
-        b[:] = 0.0
-    elif kind == "precision_sum":       # a = 1, p = 0: lambda is a running sum of phi
-        a[:] = 1.0
-        p[:] = 0.0
-    elif kind == "negative_decay":      # the gate follows the sign of a
-        a *= np.where(rng.random(sh) < 0.5, -1.0, 1.0)
-    elif kind == "mixed_zeros":         # some tokens without noise, some without evidence
-        p[rng.random(sh) < 0.3] = 0.0
-        z = rng.random(sh) < 0.3
-        phi[z] = 0.0
-        b[z] = 0.0
-    x = {k: v.astype(np.float32) for k, v in (("a", a), ("p", p), ("phi", phi), ("b", b))}
-    x["lam0"] = rng.uniform(0.5, 2.0, (B, H, N)).astype(np.float32)
-    x["eta0"] = rng.standard_normal((B, H, N)).astype(np.float32)
-    return x
-
-
-SPECIAL = ["no_process_noise", "no_observation", "precision_sum", "negative_decay", "mixed_zeros"]
+SPECIAL = wl.SPECIAL_CASES
+_special_inputs = wl.special_inputs
 
 
 @pytest.mark.parametrize("kind", SPECIAL)
