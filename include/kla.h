@@ -46,7 +46,9 @@
  * - Preconditions, not checked per element: p_t >= 0, phi_t >= 0,
  *   lambda_0 > 0, and a_t^2 + p_t lambda_{t-1} > 0 (e.g. a_t != 0 or p_t > 0).
  *   Any real a_t is allowed (only a_t^2 enters the precision; the sign of a_t
- *   enters the gate).
+ *   enters the gate).  The state must stay within fp32 range: with p_t = 0
+ *   and |a_t| < 1 the precision grows like a^(-2t) and overflows after about
+ *   44 / -ln|a| tokens (the fp64 oracle goes further).
  * - Arithmetic: inputs are fp32 or bf16 (converted exactly to fp32 on load);
  *   state, arithmetic and outputs are fp32 (the gradients of an input are
  *   written in that input's dtype); reciprocals use the hardware instruction
