@@ -42,6 +42,7 @@ from kalman_linear_attention_b200 import workloads as wl  # noqa: E402
 METRIC = "scan throughput (token-channels/s) and achieved HBM GB/s vs B200 peak, 1 GPU"
 UNIT = "token-channels/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (context beside the measured peak)
 CSRC = os.path.join(ROOT, "kalman_linear_attention_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
@@ -554,6 +555,7 @@ def run_ours(args):
         "gb_per_s": bpt * tc_all * args.steps / (max_ms * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
+                     "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                      "traffic": traffic, "algorithmic_bytes_per_launch": bpt * tc_rank,
                      "kernel": kernel_name, "launch_ms": launch_ms},
         "gpu_launches": plan[1] * args.steps,
