@@ -51,3 +51,40 @@ def test_bf16_rounding_ties_to_even():
     vals = np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9], dtype=np.float32)
     got = wl.round_to_bf16(vals)
     np.testing.assert_array_equal(got, np.array([1.0, 1.0 + 2 ** -6, 1.0], dtype=np.float32))
+
+
+def test_layer_generator_shapes_and_ranges():
+    import dataclasses
+    w = wl.LAYER_WORKLOADS["layer"].with_shape(B=2, T=40, H=2, D=6, Ns=8)
+    x = wl.generate_layer(w)
+    assert x["k"].shape == (2, 40, 2, 8) and x["v"].shape == (2, 40, 2, 6) and x["a"].shape == (2, 6, 8)
+    assert np.all(x["w"] > 0) and np.all((x["a"] > 0) & (x["a"] < 1)) and np.all(x["p"] > 0)
+    # bf16 workloads carry bf16-representable values
+    assert np.array_equal(wl.round_to_bf16(x["k"]), x["k"])
+    y = wl.generate_layer(w)
+    assert all(np.array_equal(x[k], y[k]) for k in x)                    # seeded
+    f32 = wl.generate_layer(dataclasses.replace(w, dtype="f32"))
+    assert not np.array_equal(wl.round_to_bf16(f32["v"]), f32["v"])      # fp32 keeps its bits
+    pr = wl.random_layer_prior(w)
+    assert pr["lam0"].shape == (2, 2, 6, 8) and np.all(pr["lam0"] > 0)
+
+
+def test_output_gradients_do_not_depend_on_block_size():
+    w = wl.WORKLOADS["tiny"].with_shape(B=2, T=30, H=1, N=8)
+    full = wl.generate_output_grads(w)
+    parts = list(wl.iter_output_grad_rows(w, rows_per_block=7))
+    for k in wl.GRAD_NAMES:
+        cat = np.concatenate([blk[k] for _, _, blk in parts]).reshape(full[k].shape)
+        assert np.array_equal(cat, full[k]), k
+
+
+@pytest.mark.parametrize("kind", wl.SPECIAL_CASES)
+def test_special_inputs(kind):
+    x = wl.special_inputs(kind, T=50)
+    assert np.all(x["p"] >= 0) and np.all(x["phi"] >= 0) and np.all(x["lam0"] > 0)
+    if kind in ("no_process_noise", "precision_sum"):
+        assert np.all(x["p"] == 0)
+    if kind == "no_observation":
+        assert np.all(x["phi"] == 0) and np.all(x["b"] == 0)
+    if kind == "precision_sum":
+        assert np.all(x["a"] == 1)
