@@ -5,10 +5,13 @@ the CPU-baseline / reference legs of ``bench.py`` may import this package.  The
 product path (``kalman_linear_attention_b200``) never imports it, and this
 package never imports the product path: the two share no code.
 
-The arithmetic lives in ``kla_oracle.c`` (plain sequential covariance-form
-Kalman filter, fp64, one channel at a time).  This module only compiles it with
-gcc, loads it with ctypes and converts arrays to contiguous fp64 (an exact
-upcast for fp32 and bf16 inputs).
+The filter's arithmetic lives in ``kla_oracle.c`` (plain sequential
+covariance-form Kalman filter and its reverse-mode gradients, fp64, one channel
+at a time).  This module compiles it with gcc, loads it with ctypes and
+converts arrays to contiguous fp64 (an exact upcast for fp32 and bf16 inputs).
+The one piece of arithmetic written here is the KLA layer around the filter
+(``layer_forward``): the evidence formed from the layer's operators by numpy
+broadcasting, and the readout by sums over the state channels, in fp64.
 
 Pins: every function here is pinned by ``tests/test_oracle.py`` against exact
 rational arithmetic, closed forms (Riccati fixed point, precision sums, the
@@ -17,7 +20,9 @@ invariants.  The gradients (``backward``, reverse mode through the covariance
 form) are pinned against exact forward-mode derivatives (dual numbers over
 Fractions) of the exact Moebius/affine filter, torch autograd through the
 information form, central finite differences of the pinned forward pass, and
-closed-form sums of the a = 1 / p = 0 cases.  None is "parity unpinned".
+closed-form sums of the a = 1 / p = 0 cases.  The layer function is pinned
+against exact rationals computed channel by channel with plain loops and
+against one-hot readouts of the pinned filter.  None is "parity unpinned".
 """
 from __future__ import annotations
 
