@@ -206,3 +206,25 @@ def test_layer_step_host_argument_errors(lib):
     assert f(*args(y=P)) == 1          # y overlaps k
     assert f(*args(eta=7 * P)) == 1    # state halves overlap
     assert f(*args(B=0)) == 0
+
+
+def test_header_is_plain_c(lib, tmp_path):
+    """include/kla.h compiles as strict C99 (a C caller can use the ABI) and
+    its prototypes match the library's exports in a C program that takes the
+    address of every function."""
+    import subprocess
+    names = declared_functions()
+    src = tmp_path / "use.c"
+    src.write_text('#include "kla.h"\ntypedef void (*any_fn)(void);\nint main(void) {\n    int n = 0;\n'
+                   + "".join(f"    n += (any_fn){n} != (any_fn)0;\n" for n in names)
+                   + f"    return n == {len(names)} && kla_abi_version() == KLA_ABI_VERSION ? 0 : 1;\n}}\n")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    # link a C program against the library and run it (no CUDA call is made)
+    pkg = os.path.dirname(lib._name)
+    exe = tmp_path / "use"
+    r = subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", pkg, "-l:libkla.so", f"-Wl,-rpath,{pkg}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
