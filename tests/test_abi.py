@@ -228,3 +228,23 @@ def test_header_is_plain_c(lib, tmp_path):
                         "-L", pkg, "-l:libkla.so", f"-Wl,-rpath,{pkg}"], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_size_overflow_is_rejected(lib):
+    """Sizes whose products overflow int64 are argument errors, answered on
+    the host for every entry point that takes a shape."""
+    P = 1 << 20
+    big = 1 << 40
+    assert lib.kla_scan_forward(P, 2 * P, 3 * P, 4 * P, 0, 5 * P, 6 * P, 7 * P, 8 * P, None, None,
+                                big, big, 1, 1, 16 * P, 1 << 20, None) == 1
+    out = ctypes.c_size_t(0)
+    assert lib.kla_scan_forward_workspace_size(big, big, 1, 1, 0, ctypes.byref(out)) == 1
+    assert lib.kla_scan_backward_workspace_size(1, big, big, 1, 0, ctypes.byref(out)) == 1
+    assert lib.kla_scan_backward(P, 2 * P, 0, 3 * P, 4 * P, 5 * P, 6 * P, None, None, None, None,
+                                 7 * P, 8 * P, 9 * P, 10 * P, 11 * P, 12 * P, big, big, 1, 1,
+                                 16 * P, 1 << 20, None) == 1
+    assert lib.kla_scan_step(P, 2 * P, 3 * P, 4 * P, 0, 5 * P, 6 * P, None, None, big, big, 1, None) == 1
+    assert lib.kla_layer_forward(P, 2 * P, 3 * P, 4 * P, 0, 5 * P, 6 * P, 7 * P, 8 * P, 9 * P, None, None, None,
+                                 big, big, 1, 2, 16, 16 * P, 1 << 20, None) == 1
+    assert lib.kla_layer_step(P, 2 * P, 3 * P, 4 * P, 0, 5 * P, 6 * P, 7 * P, 8 * P, 9 * P, None,
+                              big, big, 2, 16, None) == 1
