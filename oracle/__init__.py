@@ -22,7 +22,10 @@ Fractions) of the exact Moebius/affine filter, torch autograd through the
 information form, central finite differences of the pinned forward pass, and
 closed-form sums of the a = 1 / p = 0 cases.  The layer function is pinned
 against exact rationals computed channel by channel with plain loops and
-against one-hot readouts of the pinned filter.  None is "parity unpinned".
+against one-hot readouts of the pinned filter; its gradients
+(``layer_backward``, not yet matched by a kernel) against exact forward-mode
+derivatives of the exact layer and finite differences of the pinned layer
+function.  None is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -216,6 +219,80 @@ class Oracle:
             lam_T, eta_T = lam0.copy(), eta0.copy()
         return {"y": y, "s": s_, "lam_T": lam_T, "eta_T": eta_T}
 
+    def layer_backward(self, k, q, v, w, a, p, lam0, eta0, g_y=None, g_s=None, g_lam_T=None, g_eta_T=None,
+                       threads: int = 1):
+        """Gradients of a loss through ``layer_forward``.
+
+        ``g_y``, ``g_s`` [B, T, H, D] and ``g_lam_T``, ``g_eta_T``
+        [B, H, D, Ns] are the loss gradients with respect to the layer's
+        outputs (None: zero).  Returns fp64 gradients with respect to every
+        input: ``k``, ``q``, ``v``, ``w``, ``a``, ``p``, ``lam0``, ``eta0``.
+
+        The chain rule over the layer's three parts: the readout (d y / d mu =
+        q_n, d s / d var = q_n^2, d y / d q_n = mu, d s / d q_n = 2 q_n var), the
+        filter (the reverse-mode ``backward`` of the C oracle, with the final
+        state's gradients added at the last token), and the evidence (phi =
+        k^2 w, b = k w v; a and p are shared by every token and batch row, so
+        their gradients are sums).
+        """
+        k, q, v, w = (_f64(x) for x in (k, q, v, w))
+        a, p = _f64(a), _f64(p)
+        B, T, H, Ns = k.shape
+        D = v.shape[3]
+        shape5 = (B, T, H, D, Ns)
+        lam0 = _f64(np.broadcast_to(np.asarray(lam0, dtype=np.float64), (B, H, D, Ns)))
+        eta0 = _f64(np.broadcast_to(np.asarray(eta0, dtype=np.float64), (B, H, D, Ns)))
+        zero4 = np.zeros((B, T, H, D))
+        g_y = zero4 if g_y is None else _f64(g_y)
+        g_s = zero4 if g_s is None else _f64(g_s)
+        kk = k[:, :, :, None, :]
+        ww = w[:, :, :, :, None]
+        vv = v[:, :, :, :, None]
+        qq = q[..., None, :]
+        phi = ww * (kk * kk)                  # the forward's evidence, recomputed
+        info = (kk * vv) * ww
+        flat = lambda x: np.ascontiguousarray(np.broadcast_to(x, shape5)).reshape(B, T, H, D * Ns)
+        fwd = self.forward(flat(a), flat(p), flat(phi), flat(info), lam0.reshape(B, H, D * Ns),
+                           eta0.reshape(B, H, D * Ns), threads=threads)
+        mu = fwd["mu"].reshape(shape5)
+        var = fwd["var"].reshape(shape5)
+        # readout
+        g_mu = g_y[..., None] * qq
+        g_var = g_s[..., None] * qq * qq
+        g_q = np.sum(g_y[..., None] * mu + 2.0 * g_s[..., None] * qq * var, axis=3)
+        # final state -> gradients of the last row of lambda, eta
+        g_lam = np.zeros(shape5)
+        g_eta = np.zeros(shape5)
+        if T > 0:
+            if g_lam_T is not None:
+                g_lam[:, T - 1] = _f64(g_lam_T)
+            if g_eta_T is not None:
+                g_eta[:, T - 1] = _f64(g_eta_T)
+        gr = self.backward(flat(a), flat(p), flat(phi), flat(info), lam0.reshape(B, H, D * Ns),
+                           eta0.reshape(B, H, D * Ns), flat(g_lam), flat(g_eta), flat(g_mu), flat(g_var),
+                           threads=threads)
+        g_phi = gr["phi"].reshape(shape5)
+        g_b = gr["b"].reshape(shape5)
+        out = {
+            # evidence: phi = k^2 w, b = k w v
+            "k": np.sum(g_phi * 2.0 * kk * ww + g_b * ww * vv, axis=3),
+            "w": np.sum(g_phi * kk * kk + g_b * kk * vv, axis=4),
+            "v": np.sum(g_b * kk * ww, axis=4),
+            "q": g_q,
+            # time-invariant parameters: summed over batch rows and tokens
+            "a": np.sum(gr["a"].reshape(shape5), axis=(0, 1)),
+            "p": np.sum(gr["p"].reshape(shape5), axis=(0, 1)),
+            "lam0": gr["lam0"].reshape(B, H, D, Ns),
+            "eta0": gr["eta0"].reshape(B, H, D, Ns),
+        }
+        if T == 0:
+            # no tokens: the final state is the prior
+            if g_lam_T is not None:
+                out["lam0"] = out["lam0"] + _f64(g_lam_T)
+            if g_eta_T is not None:
+                out["eta0"] = out["eta0"] + _f64(g_eta_T)
+        return out
+
 
 _DEFAULT: Oracle | None = None
 
@@ -243,3 +320,8 @@ def backward(a, p, phi, b, lam0, eta0, g_lam=None, g_eta=None, g_mu=None, g_var=
 
 def layer_forward(k, q, v, w, a, p, lam0, eta0, threads: int = 1):
     return default().layer_forward(k, q, v, w, a, p, lam0, eta0, threads=threads)
+
+
+def layer_backward(k, q, v, w, a, p, lam0, eta0, g_y=None, g_s=None, g_lam_T=None, g_eta_T=None,
+                   threads: int = 1):
+    return default().layer_backward(k, q, v, w, a, p, lam0, eta0, g_y, g_s, g_lam_T, g_eta_T, threads=threads)

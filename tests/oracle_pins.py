@@ -653,7 +653,92 @@ def pin_layer_one_hot_readout(orc):
     _rel_close(g3["s"], 9.0 * g1["s"], 1e-14, "variance readout quadratic in q")
 
 
-LAYER_PINS = [pin_layer_exact, pin_layer_one_hot_readout]
+def _exact_layer_loss(fr, w4):
+    """Exact loss sum g_y y + g_s s + g_lamT lam_T + g_etaT eta_T of the layer,
+    channel by channel with plain loops, on Fraction or Dual entries."""
+    g_y, g_s, g_lT, g_eT = w4
+    B, T, H, Ns = fr["k"].shape
+    D = fr["v"].shape[3]
+    tot = Fr(0)
+    for bi in range(B):
+        for h in range(H):
+            for d in range(D):
+                for n in range(Ns):
+                    phi = [fr["k"][bi, t, h, n] * fr["k"][bi, t, h, n] * fr["w"][bi, t, h, d] for t in range(T)]
+                    info = [fr["k"][bi, t, h, n] * fr["w"][bi, t, h, d] * fr["v"][bi, t, h, d] for t in range(T)]
+                    lam, eta = exact_moebius_filter([fr["a"][h, d, n]] * T, [fr["p"][h, d, n]] * T, phi, info,
+                                                    fr["lam0"][bi, h, d, n], fr["eta0"][bi, h, d, n])
+                    for t in range(T):
+                        qq = fr["q"][bi, t, h, n]
+                        tot = tot + g_y[bi, t, h, d] * (qq * (eta[t] / lam[t])) + g_s[bi, t, h, d] * (qq * qq / lam[t])
+                    tot = tot + g_lT[bi, h, d, n] * lam[-1] + g_eT[bi, h, d, n] * eta[-1]
+    return tot
+
+
+def pin_layer_backward_exact_dual(orc, seed=51):
+    """Layer gradients == exact forward-mode derivatives (Dual numbers over
+    Fractions) of the exact layer, for every element of every input
+    (B = 2, T = 3, H = 1, D = 2, Ns = 2), with gradients on all four outputs."""
+    fr = random_rational_layer(seed, B=2, T=3, H=1, D=2, Ns=2)
+    rng = np.random.default_rng(seed + 7)
+    def rarr(shape):
+        x = np.empty(shape, dtype=object)
+        for idx in np.ndindex(shape):
+            x[idx] = _random_fraction(rng, -5, 5, 4)
+        return x
+    B, T, H, Ns = fr["k"].shape
+    D = fr["v"].shape[3]
+    w4 = (rarr((B, T, H, D)), rarr((B, T, H, D)), rarr((B, H, D, Ns)), rarr((B, H, D, Ns)))
+    exact = {}
+    for key, arr in fr.items():
+        g = np.empty(arr.shape, dtype=object)
+        for idx in np.ndindex(arr.shape):
+            dual = {kk: np.vectorize(Dual, otypes=[object])(vv) for kk, vv in fr.items()}
+            dual[key][idx] = Dual(arr[idx], 1)
+            g[idx] = _exact_layer_loss(dual, w4).d
+        exact[key] = g
+    f64 = {kk: _to_f64(vv) for kk, vv in fr.items()}
+    got = orc.layer_backward(f64["k"], f64["q"], f64["v"], f64["w"], f64["a"], f64["p"], f64["lam0"], f64["eta0"],
+                             *[_to_f64(x) for x in w4])
+    for key in exact:
+        ref = _to_f64(exact[key])
+        _scaled_close(got[key].reshape(-1), ref.reshape(-1), 1e-12, f"exact layer gradient d/d{key}", axis=None)
+
+
+def pin_layer_backward_finite_difference(orc):
+    """Layer gradients == central finite differences of the pinned layer
+    forward, sampled elements of every input, workload-like values."""
+    import dataclasses
+    rng = np.random.default_rng(61)
+    w = dataclasses.replace(wl.LAYER_WORKLOADS["layer"].with_shape(B=2, T=20, H=2, D=2, Ns=8), dtype="f32")
+    x = {kk: np.asarray(vv, dtype=np.float64) for kk, vv in wl.generate_layer(w).items()}
+    x.update({kk: np.asarray(vv, dtype=np.float64) for kk, vv in wl.random_layer_prior(w).items()})
+    gw = (rng.standard_normal((w.B, w.T, w.H, w.D)), rng.standard_normal((w.B, w.T, w.H, w.D)),
+          rng.standard_normal((w.B, w.H, w.D, w.Ns)), rng.standard_normal((w.B, w.H, w.D, w.Ns)))
+    names = ("k", "q", "v", "w", "a", "p", "lam0", "eta0")
+    got = orc.layer_backward(*(x[n] for n in names), *gw)
+
+    def loss(arrs):
+        o = orc.layer_forward(*(arrs[n] for n in names))
+        return math.fsum(float((g * o[kk]).sum()) for g, kk in zip(gw, ("y", "s", "lam_T", "eta_T")))
+
+    for key in names:
+        for _ in range(4):
+            idx = tuple(int(rng.integers(0, s_)) for s_ in x[key].shape)
+            h = 1e-6 * max(abs(x[key][idx]), 1e-2)
+            up = dict(x)
+            dn = dict(x)
+            up[key] = x[key].copy()
+            dn[key] = x[key].copy()
+            up[key][idx] += h
+            dn[key][idx] -= h
+            fd = (loss(up) - loss(dn)) / (2 * h)
+            g = got[key][idx]
+            assert abs(g - fd) <= 2e-5 * (abs(fd) + 1e-2), f"layer d/d{key}{idx}: {g} vs finite difference {fd}"
+
+
+LAYER_PINS = [pin_layer_exact, pin_layer_one_hot_readout, pin_layer_backward_exact_dual,
+              pin_layer_backward_finite_difference]
 
 BACKWARD_PINS = [pin_backward_exact_dual, pin_backward_autograd, pin_backward_finite_difference,
                  pin_backward_closed_forms]

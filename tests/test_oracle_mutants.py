@@ -82,6 +82,16 @@ LAYER_MUTANTS = {
     "layer: final state from the first token": ('lam_T = out["lam"][:, T - 1]', 'lam_T = out["lam"][:, 0]'),
     "layer: k read out instead of q": ("qq = q[:, :, :, None, :]", "qq = k[:, :, :, None, :]"),
     "layer: a and p swapped": ("self.forward(flat(aa), flat(pp),", "self.forward(flat(pp), flat(aa),"),
+    "layer backward: dk without the factor 2": ("g_phi * 2.0 * kk * ww", "g_phi * kk * ww"),
+    "layer backward: dw with k, not k^2": ("g_phi * kk * kk + g_b * kk * vv", "g_phi * kk + g_b * kk * vv"),
+    "layer backward: dq without the variance term": (
+        "np.sum(g_y[..., None] * mu + 2.0 * g_s[..., None] * qq * var, axis=3)",
+        "np.sum(g_y[..., None] * mu, axis=3)"),
+    "layer backward: da from the first batch row": ('"a": np.sum(gr["a"].reshape(shape5), axis=(0, 1)),',
+                                                    '"a": np.sum(gr["a"].reshape(shape5), axis=1)[0],'),
+    "layer backward: final precision gradient dropped": ("g_lam[:, T - 1] = _f64(g_lam_T)", "pass"),
+    "layer backward: variance readout gradient with q": ("g_var = g_s[..., None] * qq * qq",
+                                                          "g_var = g_s[..., None] * qq"),
 }
 
 
