@@ -224,6 +224,95 @@ def time_forward(kla, w, dev, steps: int, warmup: int, dist_mod):
     return total_ms, per_launch, plan, outs
 
 
+L2_FLUSH_BYTES = 256 << 20  # twice the B200's 126 MB L2
+
+
+def l2_flusher(device):
+    """A function that overwrites a buffer twice the size of L2 (evicting
+    whatever the previous launch left there), to be called between timed
+    launches, outside the events."""
+    import torch
+    buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+
+    def flush():
+        buf.fill_(0)
+    return flush
+
+
+def time_launches(fn, steps: int, warmup: int, flush=None):
+    """Per-launch CUDA-event times (ms) of `fn` on the current stream: `warmup`
+    untimed calls, then `steps` calls each bracketed by its own events, the L2
+    flushed before each one (outside the events) when `flush` is given."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        if flush is not None:
+            flush()
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+FORWARD_KERNELS = {1: "kla_forward_kernel (chunked, cross-CTA carries; + its workspace clear kernel)",
+                   2: "kla_forward_stream_kernel (channel-owning streaming)"}
+
+
+def time_config(kla, w: wl.Workload, device, steps: int, warmup: int, peak: float, flush):
+    """One forward workload timed on its own: the median of `steps` per-launch
+    CUDA-event times of kla_scan_forward (every output written), the L2
+    flushed between launches.  Returns the entry of the bench line's
+    ``configs`` object (without the CPU baseline) and the host arrays."""
+    import torch
+    x = wl.generate(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    d = {k: torch.from_numpy(x[k]).to(device=device, dtype=dt) for k in wl.INPUT_NAMES}
+    for k in ("lam0", "eta0"):
+        d[k] = torch.from_numpy(x[k]).to(device)
+    outs = [torch.empty((w.B, w.T, w.H, w.N), dtype=torch.float32, device=device) for _ in range(4)]
+    ws = kla.new_workspace(w.B, w.T, w.H, w.N, dt, device)
+    plan = kla.forward_plan(d["a"], d["p"], d["phi"], d["b"])
+    args = (d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    per = time_launches(lambda: kla.scan_forward(*args, out=outs, workspace=ws), steps, warmup, flush)
+    if kla.get_error() != 0:
+        raise RuntimeError(f"device-side error while timing {w.name}")
+    ms = statistics.median(per)
+    tc = w.token_channels
+    bpt = algorithmic_bytes_per_tc(w)
+    gbs = bpt * tc / (ms * 1e-3) / 1e9
+    del d, outs, ws
+    entry = {"workload": w.summary, "B": w.B, "H": w.H, "N": w.N, "T": w.T, "dtype": w.dtype,
+             "ms": ms, "ms_min": min(per), "ms_max": max(per), "launches_timed": steps, "warmup": warmup,
+             "value": tc / (ms * 1e-3), "unit": UNIT, "gb_per_s": gbs,
+             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                          "frac_of_nominal": gbs / NOMINAL_HBM_GBS,
+                          "algorithmic_bytes_per_launch": bpt * tc, "bytes_per_token_channel": bpt},
+             "kernel": FORWARD_KERNELS[plan[0]], "launches_per_call": plan[1],
+             "timing": "median of per-launch CUDA events, L2 flushed (256 MB write) between launches"}
+    return entry, x
+
+
+def time_copy_bandwidth(device, steps: int = 20, nbytes: int = 4 << 30):
+    """Device-to-device copy bandwidth of this GPU in this run: read + write
+    bytes of a 4 GiB torch copy over the median CUDA-event time.  It is
+    context for the roofline fractions (boxes differ), not their denominator."""
+    import torch
+    src = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+    src.fill_(1.0)
+    dst = torch.empty_like(src)
+    per = time_launches(lambda: dst.copy_(src), steps, 3)
+    ms = statistics.median(per)
+    del src, dst
+    return {"gb_per_s": 2 * nbytes / (ms * 1e-3) / 1e9, "ms": ms,
+            "how": "torch copy_ of a 4 GiB fp32 buffer on the device, (read + write bytes) / median of "
+                   f"{steps} CUDA-event times"}
+
+
 def backward_bytes_per_tc(w: wl.Workload) -> int:
     """Bytes the backward scan must move per token-channel with all four
     output gradients present: read a, p (input dtype), lambda, eta and the
@@ -262,7 +351,7 @@ def time_backward(kla, w, dev, outs, steps: int, warmup: int, peak: float, traff
     torch.cuda.synchronize()
     if kla.get_error() != 0:
         raise RuntimeError("device-side error in the timed backward region")
-    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
     bpt = backward_bytes_per_tc(w)
     tc = w.token_channels
     gbs = bpt * tc / (ms * 1e-3) / 1e9
@@ -332,8 +421,10 @@ def time_decode(kla, device, steps_tokens: int | None, replays: int):
     del g
     tc = w.channels
     bytes_step = decode_bytes_per_channel(w) * tc
+    in_bytes = (2 if w.dtype == "bf16" else 4) * 4 * tc
     return {"workload": w.summary, "ms_per_token": ms, "value": tc / (ms * 1e-3), "unit": UNIT,
             "gb_per_s": bytes_step / (ms * 1e-3) / 1e9, "bytes_per_token": bytes_step,
+            "input_bytes_per_token": in_bytes, "input_gb_per_s": in_bytes / (ms * 1e-3) / 1e9,
             "tokens_per_replay": w.T, "replays": replays,
             "note": "one kla_scan_step launch per token; the 8 MB fp32 state can stay L2-resident"}
 
@@ -385,7 +476,7 @@ def time_layer(kla, device, steps: int, warmup: int):
         torch.cuda.synchronize()
         if kla.get_error() != 0:
             raise RuntimeError("device-side error in the timed layer region")
-        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
 
     ms = timed(fused, steps)
     ms_unfused = timed(unfused, max(3, steps // 10))
@@ -438,12 +529,12 @@ def time_layer(kla, device, steps: int, warmup: int):
                     "a, p and reading out, kla_scan_forward in between) moves about 40 B per token-channel"}
 
 
-def cpu_oracle_sample(w: wl.Workload, host_arrays, target_s: float = 10.0):
-    """Time the fp64 oracle on a bounded sample of whole channels of the workload."""
+def cpu_oracle_sample(w: wl.Workload, host_arrays, target_s: float = 10.0, threads: int | None = None):
+    """Time the fp64 oracle on a bounded sample of whole channels of the
+    workload, on `threads` host threads (default: every core)."""
     import oracle
-    threads = os.cpu_count() or 1
     orc = oracle.default()
-    threads = min(threads, orc.max_threads())
+    threads = min(threads or os.cpu_count() or 1, orc.max_threads())
     HN = w.H * w.N
 
     def run(nch):
@@ -461,9 +552,14 @@ def cpu_oracle_sample(w: wl.Workload, host_arrays, target_s: float = 10.0):
     while dt < target_s / 4 and n < w.channels:
         n = min(w.channels, int(n * max(2.0, target_s / max(dt, 1e-3) / 2)))
         dt = run(n)
+    reps = 1
+    if dt < target_s / 4:  # the whole workload is a small sample: repeat it
+        reps = max(1, min(1000, int(target_s / 4 / max(dt, 1e-6))))
+        dt = min(sum(run(n) for _ in range(reps)) / reps for _ in range(2))
     return {"value": n * w.T / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n} of {w.channels} channels x all {w.T} tokens ({n * w.T:,} token-channels), "
-                      f"fp64 sequential covariance-form filter, OpenMP over channels, {dt:.2f} s"}
+            "sample": f"{n} of {w.channels} channels x all {w.T} tokens ({n * w.T:,} token-channels)"
+                      + (f", best of 2 means of {reps} runs" if reps > 1 else "")
+                      + f", fp64 sequential covariance-form filter, OpenMP over channels, {dt:.3g} s per run"}
 
 
 def run_ours(args):
@@ -502,7 +598,7 @@ def run_ours(args):
     tc_all = tc_rank * world
     value = tc_all * args.steps / (max_ms * 1e-3)
     bpt = algorithmic_bytes_per_tc(w)
-    launch_ms = statistics.mean(per_launch)
+    launch_ms = statistics.median(per_launch)
     achieved = bpt * tc_rank / (launch_ms * 1e-3) / 1e9
     peak, peak_src = measured_peaks()
     traffic = recorded_traffic(args.workload if not args.tokens else f"{args.workload}@T={args.tokens}",
@@ -532,12 +628,53 @@ def run_ours(args):
     decode = None
     if not args.no_decode:
         decode = time_decode(kla, device, None, args.decode_replays)
-        decode["gb_per_s_frac_of_peak"] = decode["gb_per_s"] / peak
+        decode["input_roofline"] = {
+            "bound": "hbm", "achieved": decode["input_gb_per_s"], "peak": peak, "unit": "GB/s",
+            "frac": decode["input_gb_per_s"] / peak,
+            "note": "the token inputs (a, p, phi, b) are the only bytes that must come from HBM each step; "
+                    "the state and the mu / var buffers stay L2-resident between steps"}
+
+    # every forward workload of the task timed on its own (one GPU only)
+    configs = None
+    copy_bw = None
+    if world == 1 and not args.no_configs:
+        flush = l2_flusher(device)
+        configs = {}
+        host_cfg = {}
+        for name in ("tiny", "lm_layer", "stiff"):
+            configs[name], host_cfg[name] = time_config(kla, wl.WORKLOADS[name], device, args.config_steps,
+                                                        args.warmup, peak, flush)
+        configs["long"] = {
+            "workload": base.summary, "B": base.B, "H": base.H, "N": base.N, "T": base.T, "dtype": base.dtype,
+            "ms": launch_ms, "ms_min": min(per_launch), "ms_max": max(per_launch),
+            "launches_timed": len(per_launch), "warmup": args.warmup, "value": tc_rank / (launch_ms * 1e-3),
+            "unit": UNIT, "gb_per_s": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                         "algorithmic_bytes_per_launch": bpt * tc_rank, "bytes_per_token_channel": bpt},
+            "kernel": kernel_name, "launches_per_call": plan[1],
+            "timing": "the headline's timed steps: median of per-launch CUDA events, back to back "
+                      "(inputs of 4.3 GB, larger than L2)"}
+        del flush
+        torch.cuda.empty_cache()
+        copy_bw = time_copy_bandwidth(device)
+        for e in configs.values():
+            e["roofline"]["frac_of_same_run_copy"] = e["gb_per_s"] / copy_bw["gb_per_s"]
+        if rank == 0 and not args.no_cpu_baseline:
+            for name in ("tiny", "lm_layer", "stiff"):
+                w_c = wl.WORKLOADS[name]
+                configs[name]["cpu_baseline"] = cpu_oracle_sample(w_c, host_cfg[name], args.cpu_target_s)
+                configs[name]["cpu_baseline_1core"] = cpu_oracle_sample(w_c, host_cfg[name], args.cpu_target_s,
+                                                                        threads=1)
+        del host_cfg
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and host is not None:
         arrays = {k: host[k].float().numpy() for k in wl.INPUT_NAMES}
         cpu = cpu_oracle_sample(w, arrays)
+        if configs is not None:
+            configs["long"]["cpu_baseline"] = cpu
+            configs["long"]["cpu_baseline_1core"] = cpu_oracle_sample(w, arrays, args.cpu_target_s, threads=1)
 
     if world > 1:
         dist.barrier()
@@ -564,6 +701,8 @@ def run_ours(args):
         "decode": decode,
         "backward": backward,
         "layer": layer,
+        "configs": configs,
+        "hbm_copy_same_run": copy_bw,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line))
@@ -625,6 +764,11 @@ def parse_args(argv=None):
     ap.add_argument("--backward-steps", type=int, default=50)
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--layer-steps", type=int, default=50)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the tiny, LM-layer and stiff workloads on their own")
+    ap.add_argument("--config-steps", type=int, default=30)
+    ap.add_argument("--cpu-target-s", type=float, default=4.0,
+                    help="seconds of oracle work per CPU timing of the per-workload entries")
     return ap.parse_args(argv)
 
 

@@ -175,8 +175,12 @@ kla_status_t kla_debug_force_forward_kernel(int which);
  *   N=128); larger problems return KLA_ERR_TOO_LARGE before anything is
  *   enqueued.
  * - First call on a device: it looks up the device address of the static
- *   array (cudaGetSymbolAddress) with that device current, and caches it.
- *   Make that first call before any stream capture begins.
+ *   array (cudaGetSymbolAddress) with that device current, and caches it for
+ *   the life of the process.  Make that first call before any stream capture
+ *   begins.  cudaDeviceReset unloads the library's device code with the
+ *   context, and the array may sit elsewhere afterwards while the cached
+ *   address does not change: a process that resets a device must not call
+ *   this entry point on that device again.
  * - Sharing: every call on a device uses the same array, which keeps what the
  *   last call left in it; each call re-zeroes, on its stream, the part that
  *   must start at zero.  Calls whose work overlaps on the GPU (two streams,

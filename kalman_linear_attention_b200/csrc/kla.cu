@@ -385,7 +385,7 @@ KLA_API kla_status_t kla_scan_forward_workspace_size(int64_t B, int64_t T, int64
     FwdLayout lay;
     if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
     const int64_t ntiles32 = B * ((HN + 31) / 32);
-    const StreamWs sw = stream_ws_layout(ntiles32, 4);  // the most runs the streaming kernel uses
+    const StreamWs sw = stream_ws_layout(ntiles32, KLA_STREAM_MAX_PARTS);  // the most runs stream_parts picks
     *bytes = std::max(lay.total, sw.total);
     return KLA_OK;
 }
@@ -407,12 +407,13 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
     int64_t in_bytes = 0, out_bytes = 0;
     if (!mul_ok(elems, (int64_t)esz, &in_bytes) || !mul_ok(elems, 4, &out_bytes))
         return KLA_ERR_INVALID_ARG;
-    const Range outs[4] = {range_of(lambda_out, out_bytes), range_of(eta_out, out_bytes),
-                           range_of(mu_out, out_bytes), range_of(var_out, out_bytes)};
-    const Range ins[7] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(phi, in_bytes),
-                          range_of(b, in_bytes), range_of(lambda0, C * 4), range_of(eta0, C * 4),
-                          range_of(workspace, (int64_t)workspace_bytes)};
-    if (any_overlap(outs, 4, ins, 7)) return KLA_ERR_INVALID_ARG;
+    // the workspace is written too: it may overlap no input and no output
+    const Range outs[5] = {range_of(lambda_out, out_bytes), range_of(eta_out, out_bytes),
+                           range_of(mu_out, out_bytes), range_of(var_out, out_bytes),
+                           range_of(workspace, (int64_t)workspace_bytes)};
+    const Range ins[6] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(phi, in_bytes),
+                          range_of(b, in_bytes), range_of(lambda0, C * 4), range_of(eta0, C * 4)};
+    if (any_overlap(outs, 5, ins, 6)) return KLA_ERR_INVALID_ARG;
 
     FwdLayout lay;
     if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
@@ -475,6 +476,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
             sp.part_state = nullptr;
             if (sp.parts > 1) {
                 const StreamWs sw = stream_ws_layout(sp.ntiles, sp.parts);
+                if (sw.total > workspace_bytes) return KLA_ERR_WORKSPACE_TOO_SMALL;  // size function out of step
                 sp.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
                 sp.part_state = reinterpret_cast<float *>(ws + sw.state_off);
                 if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
@@ -806,14 +808,14 @@ KLA_API kla_status_t kla_scan_backward(const void *a, const void *p, kla_dtype_t
     int64_t in_bytes = 0, f_bytes = 0, c_bytes = 0;
     if (!mul_ok(elems, (int64_t)esz, &in_bytes) || !mul_ok(elems, 4, &f_bytes) || !mul_ok(C, 4, &c_bytes))
         return KLA_ERR_INVALID_ARG;
-    const Range outs[6] = {range_of(grad_a, in_bytes), range_of(grad_p, in_bytes), range_of(grad_phi, in_bytes),
+    const Range outs[7] = {range_of(grad_a, in_bytes), range_of(grad_p, in_bytes), range_of(grad_phi, in_bytes),
                            range_of(grad_b, in_bytes), range_of(grad_lambda0, c_bytes),
-                           range_of(grad_eta0, c_bytes)};
-    const Range ins[11] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(lambda0, c_bytes),
+                           range_of(grad_eta0, c_bytes), range_of(workspace, (int64_t)workspace_bytes)};
+    const Range ins[10] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(lambda0, c_bytes),
                            range_of(eta0, c_bytes), range_of(lambda_out, f_bytes), range_of(eta_out, f_bytes),
                            range_of(g_lambda, f_bytes), range_of(g_eta, f_bytes), range_of(g_mu, f_bytes),
-                           range_of(g_var, f_bytes), range_of(workspace, (int64_t)workspace_bytes)};
-    if (any_overlap(outs, 6, ins, 11)) return KLA_ERR_INVALID_ARG;
+                           range_of(g_var, f_bytes)};
+    if (any_overlap(outs, 7, ins, 10)) return KLA_ERR_INVALID_ARG;
     size_t need = 0;
     if (kla_scan_backward_workspace_size(B, T, H, N, in_dtype, &need) != KLA_OK) return KLA_ERR_INVALID_ARG;
     if (need > 0 && (!workspace || workspace_bytes < need)) return KLA_ERR_WORKSPACE_TOO_SMALL;
@@ -866,6 +868,7 @@ KLA_API kla_status_t kla_scan_backward(const void *a, const void *p, kla_dtype_t
             prm.ticket = reinterpret_cast<unsigned *>(ws);
             if (prm.parts > 1) {
                 const StreamWs sw = stream_ws_layout(prm.ntiles, prm.parts);
+                if (sw.total > workspace_bytes) return KLA_ERR_WORKSPACE_TOO_SMALL;
                 prm.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
                 prm.part_state = reinterpret_cast<float *>(ws + sw.state_off);
                 if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
@@ -989,13 +992,13 @@ KLA_API kla_status_t kla_layer_forward(const void *k, const void *q, const void 
     const void *aligned_ins[4] = {k, q, v, w};
     for (int i = 0; i < 4; ++i)
         if (aligned_ins[i] && !aligned16(aligned_ins[i])) return KLA_ERR_INVALID_ARG;
-    const Range outs[4] = {range_of(y, vw_elems * 4), range_of(s, vw_elems * 4), range_of(lambda_T, chans * 4),
-                           range_of(eta_T, chans * 4)};
-    const Range ins[9] = {range_of(k, kq_elems * (int64_t)esz), range_of(q, kq_elems * (int64_t)esz),
+    const Range outs[5] = {range_of(y, vw_elems * 4), range_of(s, vw_elems * 4), range_of(lambda_T, chans * 4),
+                           range_of(eta_T, chans * 4), range_of(workspace, (int64_t)workspace_bytes)};
+    const Range ins[8] = {range_of(k, kq_elems * (int64_t)esz), range_of(q, kq_elems * (int64_t)esz),
                           range_of(v, vw_elems * (int64_t)esz), range_of(w, vw_elems * (int64_t)esz),
                           range_of(a, HD * Ns * 4), range_of(p, HD * Ns * 4), range_of(lambda0, chans * 4),
-                          range_of(eta0, chans * 4), range_of(workspace, (int64_t)workspace_bytes)};
-    if (any_overlap(outs, 4, ins, 9)) return KLA_ERR_INVALID_ARG;
+                          range_of(eta0, chans * 4)};
+    if (any_overlap(outs, 5, ins, 8)) return KLA_ERR_INVALID_ARG;
     size_t need = 0;
     if (kla_layer_forward_workspace_size(B, T, H, D, Ns, in_dtype, &need) != KLA_OK) return KLA_ERR_INVALID_ARG;
     if (need > 0 && (!workspace || workspace_bytes < need)) return KLA_ERR_WORKSPACE_TOO_SMALL;
@@ -1033,6 +1036,7 @@ KLA_API kla_status_t kla_layer_forward(const void *k, const void *q, const void 
     prm.ticket = reinterpret_cast<unsigned *>(ws);
     if (prm.parts > 1) {
         const StreamWs sw = stream_ws_layout(prm.ntiles, prm.parts);
+        if (sw.total > workspace_bytes) return KLA_ERR_WORKSPACE_TOO_SMALL;
         prm.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
         prm.part_state = reinterpret_cast<float *>(ws + sw.state_off);
         if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
