@@ -9,9 +9,12 @@ The filter's arithmetic lives in ``kla_oracle.c`` (plain sequential
 covariance-form Kalman filter and its reverse-mode gradients, fp64, one channel
 at a time).  This module compiles it with gcc, loads it with ctypes and
 converts arrays to contiguous fp64 (an exact upcast for fp32 and bf16 inputs).
-The one piece of arithmetic written here is the KLA layer around the filter
-(``layer_forward``): the evidence formed from the layer's operators by numpy
-broadcasting, and the readout by sums over the state channels, in fp64.
+The arithmetic written here is the KLA layer around the filter
+(``layer_forward``: the evidence formed from the layer's operators by numpy
+broadcasting, and the readout by sums over the state channels), the attention
+weights (``attention_weights``: products of the filter's gates over windows of
+tokens) and the convolutional form of the deterministic time-invariant case
+(``lti_forward``: geometric-kernel convolution sums), all in fp64.
 
 Pins: every function here is pinned by ``tests/test_oracle.py`` against exact
 rational arithmetic, closed forms (Riccati fixed point, precision sums, the
@@ -25,7 +28,13 @@ against exact rationals computed channel by channel with plain loops and
 against one-hot readouts of the pinned filter; its gradients
 (``layer_backward``, not yet matched by a kernel) against exact forward-mode
 derivatives of the exact layer and finite differences of the pinned layer
-function.  None is "parity unpinned".
+function.  The attention weights are pinned against the matrix-product
+identity prod(a) / (C lambda_s + D) of the Moebius product M_t ... M_{s+1},
+against ratios of the information mean when b = 0 after s (read off the
+pinned filter), and exact rationals; the convolutional form against the
+covariance-form filter with p = 0, exact rationals and closed forms (a = 1:
+precision sums; no evidence: geometric decay of the prior).  None is "parity
+unpinned".
 """
 from __future__ import annotations
 
@@ -219,6 +228,85 @@ class Oracle:
             lam_T, eta_T = lam0.copy(), eta0.copy()
         return {"y": y, "s": s_, "lam_T": lam_T, "eta_T": eta_T}
 
+    def attention_weights(self, a, p, phi, b, lam0, eta0, t0: int, span: int, W: int, threads: int = 1):
+        """The Kalman attention weights of the information mean, window by window.
+
+        Between two tokens s <= t of one channel, the information mean of the
+        later one responds to the earlier one through the gates between them
+        (the affine recursion eta_k = f_k eta_{k-1} + b_k, KLA review "Core
+        claim"; the "Kalman Attention Matrix" of its minor comment on
+        App. E.3/E.4):
+
+          eta_t = F(t, s) eta_s + sum_{r = s+1..t} F(t, r) b_r,
+          F(t, s) = prod_{k = s+1..t} f_k,   f_k = a_k / (a_k^2 + p_k lambda_{k-1}),
+
+        with lambda_{k-1} the posterior precision before token k (this
+        oracle's own filter; the prior before the first token).  Rows are
+        0-based tokens.  The span [t0, t0 + span) is cut into windows of W
+        tokens; returns F, fp64 [B, nwin, W, W, H, N] with nwin =
+        ceil(span / W): entry [b, w, i, j, h, n] = F(t0 + w W + i, t0 + w W + j)
+        for j <= i inside the span (1 on the diagonal), 0 above the diagonal
+        and past the span.
+        """
+        a, p = _f64(a), _f64(p)
+        if a.ndim != 4 or p.shape != a.shape:
+            raise ValueError("a, p must share one [B, T, H, N] shape")
+        B, T, H, N = a.shape
+        if W < 1 or t0 < 0 or span < 0 or t0 + span > T:
+            raise ValueError("need W >= 1 and 0 <= t0 <= t0 + span <= T")
+        lam0 = _f64(np.broadcast_to(np.asarray(lam0, dtype=np.float64), (B, H, N)))
+        out = self.forward(a, p, phi, b, lam0, eta0, threads=threads)
+        lam_before = np.concatenate([lam0[:, None], out["lam"][:, :T - 1]], axis=1)
+        gate = a / (a * a + p * lam_before)           # f_k for every token k
+        nwin = -(-span // W)
+        F = np.zeros((B, nwin, W, W, H, N))
+        for w in range(nwin):
+            start = t0 + w * W
+            n_valid = min(W, t0 + span - start)
+            for j in range(n_valid):
+                F[:, w, j, j] = 1.0
+                F[:, w, j + 1:n_valid, j] = np.cumprod(gate[:, start + j + 1:start + n_valid], axis=1)
+        return F
+
+    def lti_forward(self, a, phi, b, lam0, eta0):
+        """The convolutional form of the filter for a deterministic
+        time-invariant system (KLA review, Theorem 3: deterministic LTI
+        systems, evaluated as a convolution).
+
+        With no process noise (p = 0) and a decay a constant in time, the
+        precision map is affine, lambda_t = a^-2 lambda_{t-1} + phi_t, and
+        the gate is 1 / a, so both recursions unroll into causal
+        convolutions with geometric kernels (rows 0-based):
+
+          lambda_t = a^(-2(t+1)) lambda_0 + sum_{s=0..t} a^(-2(t-s)) phi_s,
+          eta_t    = a^(-(t+1))  eta_0    + sum_{s=0..t} a^(-(t-s))  b_s,
+
+        mu_t = eta_t / lambda_t, var_t = 1 / lambda_t.  Here the sums are
+        evaluated as written (kernel powers by ``numpy.power``, O(T^2) per
+        channel): it is the definition, for small cases.
+
+        a: [B, H, N] (per channel); phi, b: [B, T, H, N]; lam0, eta0:
+        [B, H, N].  Returns fp64 ``lam``, ``eta``, ``mu``, ``var``
+        [B, T, H, N].
+        """
+        phi, b = _f64(phi), _f64(b)
+        if phi.ndim != 4 or b.shape != phi.shape:
+            raise ValueError("phi, b must share one [B, T, H, N] shape")
+        B, T, H, N = phi.shape
+        a = _f64(np.broadcast_to(np.asarray(a, dtype=np.float64), (B, H, N)))
+        lam0 = _f64(np.broadcast_to(np.asarray(lam0, dtype=np.float64), (B, H, N)))
+        eta0 = _f64(np.broadcast_to(np.asarray(eta0, dtype=np.float64), (B, H, N)))
+        m = np.arange(T + 1, dtype=np.float64)
+        kappa = np.power(a[..., None], -2.0 * m)      # [B, H, N, T+1]: a^(-2m)
+        nu = np.power(a[..., None], -m)                # a^(-m)
+        lam = np.empty((B, T, H, N))
+        eta = np.empty((B, T, H, N))
+        for t in range(T):
+            # kernel index t - s for s = 0..t
+            lam[:, t] = kappa[..., t + 1] * lam0 + np.einsum("bhns,bshn->bhn", kappa[..., t::-1], phi[:, :t + 1])
+            eta[:, t] = nu[..., t + 1] * eta0 + np.einsum("bhns,bshn->bhn", nu[..., t::-1], b[:, :t + 1])
+        return {"lam": lam, "eta": eta, "mu": eta / lam, "var": 1.0 / lam}
+
     def layer_backward(self, k, q, v, w, a, p, lam0, eta0, g_y=None, g_s=None, g_lam_T=None, g_eta_T=None,
                        threads: int = 1):
         """Gradients of a loss through ``layer_forward``.
@@ -325,3 +413,11 @@ def layer_forward(k, q, v, w, a, p, lam0, eta0, threads: int = 1):
 def layer_backward(k, q, v, w, a, p, lam0, eta0, g_y=None, g_s=None, g_lam_T=None, g_eta_T=None,
                    threads: int = 1):
     return default().layer_backward(k, q, v, w, a, p, lam0, eta0, g_y, g_s, g_lam_T, g_eta_T, threads=threads)
+
+
+def attention_weights(a, p, phi, b, lam0, eta0, t0: int, span: int, W: int, threads: int = 1):
+    return default().attention_weights(a, p, phi, b, lam0, eta0, t0, span, W, threads=threads)
+
+
+def lti_forward(a, phi, b, lam0, eta0):
+    return default().lti_forward(a, phi, b, lam0, eta0)

@@ -740,9 +740,175 @@ def pin_layer_backward_finite_difference(orc):
 LAYER_PINS = [pin_layer_exact, pin_layer_one_hot_readout, pin_layer_backward_exact_dual,
               pin_layer_backward_finite_difference]
 
+
+# ------------------------------------------------- attention weights (gates)
+def _attention_problem(seed, B=2, T=40, H=1, N=3):
+    w = wl.WORKLOADS["tiny"].with_shape(B=B, T=T, H=H, N=N, seed=seed)
+    x = wl.generate(w)
+    x["a"] = x["a"] * np.where(np.random.default_rng(seed).random(x["a"].shape) < 0.25, -1.0, 1.0)
+    pri = wl.random_prior(w)
+    x.update(pri)
+    return {k: np.asarray(v, dtype=np.float64) for k, v in x.items()}
+
+
+def _windows(t0, span, W):
+    """(window index, first token, valid tokens) of the span cut into W-token windows."""
+    return [(w, t0 + w * W, min(W, t0 + span - (t0 + w * W))) for w in range(-(-span // W))]
+
+
+def pin_attention_moebius_product(orc):
+    """F(t, s) = prod_{k=s+1..t} a_k / (C lambda_s + D) with [[A, B], [C, D]] =
+    M_t ... M_{s+1}, numpy matrix products of the pages' M_k and lambda_s
+    from the pinned filter (the denominators of the Moebius product
+    telescope into the gates' denominators)."""
+    x = _attention_problem(41)
+    t0, span, W = 3, 30, 12
+    F = orc.attention_weights(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], t0, span, W)
+    lam = orc.forward(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"])["lam"]
+    B, T, H, N = x["a"].shape
+    assert F.shape == (B, 3, W, W, H, N), F.shape
+    for bi in range(B):
+        for n in range(N):
+            a, p, phi = (x[k][bi, :, 0, n] for k in ("a", "p", "phi"))
+            for w, start, nv in _windows(t0, span, W):
+                for j in range(W):
+                    s = start + j
+                    P = np.eye(2)
+                    for i in range(W):
+                        got = F[bi, w, i, j, 0, n]
+                        if i >= nv or j >= nv or i < j:
+                            assert got == 0.0, (bi, w, i, j, got)
+                            continue
+                        if i > j:
+                            t = start + i
+                            M = np.array([[1 + p[t] * phi[t], a[t] ** 2 * phi[t]], [p[t], a[t] ** 2]])
+                            P = M @ P
+                        ref = np.prod(a[s + 1:start + i + 1]) / (P[1, 0] * lam[bi, s, 0, n] + P[1, 1])
+                        assert abs(got - ref) <= 1e-12 * abs(ref), (bi, w, i, j, got, ref)
+
+
+def pin_attention_mean_ratio(orc):
+    """With b = 0 after token s, eta_t = F(t, s) eta_s: F read off the pinned
+    filter's information mean as eta_t / eta_s (zeroing b leaves lambda, so
+    every gate, unchanged)."""
+    x = _attention_problem(42, B=1, T=24, N=2)
+    t0, span, W = 2, 20, 7
+    F = orc.attention_weights(x["a"], x["p"], x["phi"], x["b"], x["lam0"], x["eta0"], t0, span, W)
+    for w, start, nv in _windows(t0, span, W):
+        for j in range(nv):
+            s = start + j
+            bz = x["b"].copy()
+            bz[:, s + 1:] = 0.0
+            eta = orc.forward(x["a"], x["p"], x["phi"], bz, x["lam0"], x["eta0"])["eta"]
+            for i in range(j, nv):
+                ref = eta[:, start + i] / eta[:, s]
+                got = F[:, w, i, j]
+                assert np.all(np.abs(got - ref) <= 1e-12 * np.abs(ref)), (w, i, j, got, ref)
+
+
+def pin_attention_exact(orc):
+    """Exact rationals: lambda from the exact Moebius product, the gates and
+    their products in Fractions, against the fp64 weights."""
+    fr = random_rational_problem(43, B=2, T=9, H=1, N=2)
+    lam_x, _ = exact_solution(fr)
+    f64 = {k: _to_f64(v) for k, v in fr.items()}
+    t0, span, W = 1, 8, 3
+    F = orc.attention_weights(f64["a"], f64["p"], f64["phi"], f64["b"], f64["lam0"], f64["eta0"], t0, span, W)
+    B, T, H, N = fr["a"].shape
+    for bi in range(B):
+        for n in range(N):
+            lam_before = [fr["lam0"][bi, 0, n]] + list(lam_x[bi, :, 0, n])
+            gate = [fr["a"][bi, k, 0, n] / (fr["a"][bi, k, 0, n] ** 2 + fr["p"][bi, k, 0, n] * lam_before[k])
+                    for k in range(T)]
+            for w, start, nv in _windows(t0, span, W):
+                for i in range(nv):
+                    for j in range(i + 1):
+                        ref = Fr(1)
+                        for k in range(start + j + 1, start + i + 1):
+                            ref *= gate[k]
+                        got = F[bi, w, i, j, 0, n]
+                        assert abs(got - float(ref)) <= 1e-13 * abs(float(ref)), (bi, w, i, j, got, ref)
+
+
+ATTENTION_PINS = [pin_attention_moebius_product, pin_attention_mean_ratio, pin_attention_exact]
+
+
+# ------------------------------- convolutional form (deterministic, time-invariant)
+def _lti_problem(seed, B=2, T=60, H=1, N=3):
+    rng = np.random.default_rng(seed)
+    a = rng.uniform(0.9, 1.1, (B, H, N)) * np.where(rng.random((B, H, N)) < 0.3, -1.0, 1.0)
+    phi = np.exp(rng.uniform(np.log(1e-2), np.log(10.0), (B, T, H, N)))
+    b = rng.standard_normal((B, T, H, N))
+    lam0 = np.exp(rng.uniform(np.log(0.1), np.log(10.0), (B, H, N)))
+    eta0 = rng.standard_normal((B, H, N))
+    return a, phi, b, lam0, eta0
+
+
+def pin_lti_equals_filter(orc):
+    """The convolution sums equal the covariance-form filter run with p = 0
+    and the same decay at every token (Theorem 3 is a rearrangement of the
+    filter in this case)."""
+    a, phi, b, lam0, eta0 = _lti_problem(61)
+    B, T, H, N = phi.shape
+    got = orc.lti_forward(a, phi, b, lam0, eta0)
+    ref = orc.forward(np.broadcast_to(a[:, None], phi.shape), np.zeros(phi.shape), phi, b, lam0, eta0)
+    _rel_close(got["lam"], ref["lam"], 1e-12, "lti lambda")
+    _rel_close(got["var"], ref["var"], 1e-12, "lti var")
+    _scaled_close(got["eta"], ref["eta"], 1e-12, "lti eta")
+    _scaled_close(got["mu"], ref["mu"], 1e-12, "lti mu")
+
+
+def pin_lti_exact(orc):
+    """Exact rationals: the affine recursions lambda_t = a^-2 lambda_{t-1} +
+    phi_t, eta_t = eta_{t-1} / a + b_t stepped in Fractions."""
+    rng = np.random.default_rng(62)
+    B, T, H, N = 2, 10, 1, 2
+    fa = np.empty((B, H, N), dtype=object)
+    fphi = np.empty((B, T, H, N), dtype=object)
+    fb = np.empty((B, T, H, N), dtype=object)
+    for idx in np.ndindex(fa.shape):
+        fa[idx] = _random_fraction(rng, 4, 9, 7) * (-1 if rng.random() < 0.3 else 1)
+    for idx in np.ndindex(fphi.shape):
+        fphi[idx] = _random_fraction(rng, 0, 6, 8)
+        fb[idx] = _random_fraction(rng, -6, 6, 8)
+    lam0, eta0 = Fr(3, 2), Fr(-1, 3)
+    got = orc.lti_forward(_to_f64(fa), _to_f64(fphi), _to_f64(fb), float(lam0), float(eta0))
+    for idx in np.ndindex((B, H, N)):
+        bi, h, n = idx
+        lam, eta = lam0, eta0
+        for t in range(T):
+            lam = lam / (fa[idx] ** 2) + fphi[bi, t, h, n]
+            eta = eta / fa[idx] + fb[bi, t, h, n]
+            assert abs(got["lam"][bi, t, h, n] - float(lam)) <= 1e-13 * abs(float(lam)), (idx, t)
+            assert abs(got["eta"][bi, t, h, n] - float(eta)) <= 1e-13 * (abs(float(eta)) + 1), (idx, t)
+
+
+def pin_lti_closed_forms(orc):
+    """a = 1: lambda_t = lambda_0 + sum phi (math.fsum), eta_t = eta_0 + sum b;
+    no evidence (phi = b = 0): lambda_t = a^(-2(t+1)) lambda_0, eta_t =
+    a^(-(t+1)) eta_0 (the prior decays geometrically)."""
+    rng = np.random.default_rng(63)
+    T = 50
+    phi = rng.uniform(0, 3, (1, T, 1, 1))
+    b = rng.standard_normal((1, T, 1, 1))
+    got = orc.lti_forward(np.ones((1, 1, 1)), phi, b, 0.5, 0.25)
+    for t in range(T):
+        _rel_close(got["lam"][0, t, 0, 0], 0.5 + math.fsum(phi[0, :t + 1, 0, 0]), 1e-13, f"a=1 lambda t={t}")
+        ref = 0.25 + math.fsum(b[0, :t + 1, 0, 0])
+        assert abs(got["eta"][0, t, 0, 0] - ref) <= 1e-12 * (abs(ref) + 1), f"a=1 eta t={t}"
+    for a in (0.95, -1.05):
+        z = np.zeros((1, T, 1, 1))
+        got = orc.lti_forward(np.full((1, 1, 1), a), z, z, 2.0, -0.5)
+        t = np.arange(1, T + 1)
+        _rel_close(got["lam"][0, :, 0, 0], 2.0 * a ** (-2.0 * t), 1e-13, f"no-evidence lambda a={a}")
+        _rel_close(got["eta"][0, :, 0, 0], -0.5 * a ** (-1.0 * t), 1e-13, f"no-evidence eta a={a}")
+
+
+LTI_PINS = [pin_lti_equals_filter, pin_lti_exact, pin_lti_closed_forms]
+
 BACKWARD_PINS = [pin_backward_exact_dual, pin_backward_autograd, pin_backward_finite_difference,
                  pin_backward_closed_forms]
 
 ALL_PINS = [pin_exact_rational, pin_exact_rational_step, pin_riccati, pin_precision_sum,
             pin_no_process_noise, pin_no_observation, pin_gate_derivative, pin_gate_product,
-            pin_invariants] + BACKWARD_PINS + LAYER_PINS
+            pin_invariants] + BACKWARD_PINS + LAYER_PINS + ATTENTION_PINS + LTI_PINS

@@ -95,6 +95,62 @@ LAYER_MUTANTS = {
 }
 
 
+# Mistakes planted in the attention weights and the convolutional form.
+ATTENTION_MUTANTS = {
+    "attention: gate with the precision after the token": (
+        "lam_before = np.concatenate([lam0[:, None], out[\"lam\"][:, :T - 1]], axis=1)",
+        "lam_before = out[\"lam\"]"),
+    "attention: gate with a^2 on top": ("gate = a / (a * a + p * lam_before)",
+                                        "gate = a * a / (a * a + p * lam_before)"),
+    "attention: product includes the source token": (
+        "np.cumprod(gate[:, start + j + 1:start + n_valid], axis=1)",
+        "np.cumprod(gate[:, start + j:start + n_valid - 1], axis=1)"),
+    "attention: process noise dropped from the gate": ("gate = a / (a * a + p * lam_before)",
+                                                       "gate = a / (a * a + lam_before)"),
+    "attention: windows not offset by t0": ("start = t0 + w * W", "start = w * W"),
+}
+
+LTI_MUTANTS = {
+    "lti: precision kernel a^-1": ("kappa = np.power(a[..., None], -2.0 * m)",
+                                   "kappa = np.power(a[..., None], -m)"),
+    "lti: prior decayed one step short": ("lam[:, t] = kappa[..., t + 1] * lam0", "lam[:, t] = kappa[..., t] * lam0"),
+    "lti: kernel not reversed": ('np.einsum("bhns,bshn->bhn", kappa[..., t::-1], phi[:, :t + 1])',
+                                 'np.einsum("bhns,bshn->bhn", kappa[..., :t + 1], phi[:, :t + 1])'),
+    "lti: mean kernel squared": ("nu = np.power(a[..., None], -m)", "nu = np.power(a[..., None], -2.0 * m)"),
+    "lti: mu = eta lambda": ('return {"lam": lam, "eta": eta, "mu": eta / lam,',
+                             'return {"lam": lam, "eta": eta, "mu": eta * lam,'),
+}
+
+
+def _python_mutant_caught(old, new, name, pin_list):
+    import importlib.util
+    path = os.path.join(os.path.dirname(oracle.SOURCE), "__init__.py")
+    src = open(path).read()
+    assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+    spec = importlib.util.spec_from_loader("oracle_py_mutant", loader=None, origin=path)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__file__ = path
+    exec(compile(src.replace(old, new), path, "exec"), mod.__dict__)
+    orc = mod.Oracle.load(oracle.build())
+    failures = []
+    for pin in pin_list:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError, ZeroDivisionError) as e:
+            failures.append((pin.__name__, str(e)[:80]))
+    assert failures, f"no pin caught mutant {name!r}"
+
+
+@pytest.mark.parametrize("name", sorted(ATTENTION_MUTANTS))
+def test_attention_mutant_is_caught(name):
+    _python_mutant_caught(*ATTENTION_MUTANTS[name], name, pins.ATTENTION_PINS)
+
+
+@pytest.mark.parametrize("name", sorted(LTI_MUTANTS))
+def test_lti_mutant_is_caught(name):
+    _python_mutant_caught(*LTI_MUTANTS[name], name, pins.LTI_PINS)
+
+
 @pytest.mark.parametrize("name", sorted(LAYER_MUTANTS))
 def test_layer_mutant_is_caught(name):
     import importlib.util
