@@ -313,6 +313,97 @@ def time_copy_bandwidth(device, steps: int = 20, nbytes: int = 4 << 30):
                    f"{steps} CUDA-event times"}
 
 
+def time_lti(kla, device, steps: int, warmup: int, peak: float):
+    """The convolutional form (kla_scan_forward_lti) on the time-invariant
+    workload, and the general scan on the same problem (a broadcast over
+    time, p = 0) for comparison; each one's largest relative error of lambda
+    against the oracle's filter on 8 sampled whole channels."""
+    import torch
+    import oracle
+    w = wl.LTI_WORKLOADS["lti"]
+    x = wl.generate_lti(w)
+    d = {k: torch.from_numpy(x[k]).to(device) for k in ("a", "phi", "b", "lam0", "eta0")}
+    outs = [torch.empty((w.B, w.T, w.H, w.N), device=device) for _ in range(4)]
+    ws = torch.empty(max(kla.lti_workspace_size(w.B, w.T, w.H, w.N), 1), dtype=torch.uint8, device=device)
+    plan = kla.lti_plan(d["phi"], d["b"])
+    args = (d["a"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    per = time_launches(lambda: kla.scan_forward_lti(*args, out=outs, workspace=ws), steps, warmup)
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error in the convolutional form")
+    ms = statistics.median(per)
+    tc = w.token_channels
+    bpt = 2 * 4 + 4 * 4
+    gbs = bpt * tc / (ms * 1e-3) / 1e9
+    HN = w.H * w.N
+    sample = wl.channel_sample(w, 8)
+    sb, shn = np.divmod(sample, HN)
+    K = len(sample)
+    a_s = x["a"].reshape(w.B, HN)[sb, shn].reshape(1, 1, 1, K)
+    phi_s = x["phi"].reshape(w.B, w.T, HN)[sb, :, shn].T.reshape(1, w.T, 1, K)
+    b_s = x["b"].reshape(w.B, w.T, HN)[sb, :, shn].T.reshape(1, w.T, 1, K)
+    ref = oracle.forward(np.broadcast_to(a_s, phi_s.shape), np.zeros(phi_s.shape), phi_s, b_s,
+                         np.ones((1, 1, K)), np.zeros((1, 1, K)), threads=8)["lam"].reshape(w.T, K)
+
+    def lam_err(lam):
+        got = lam.view(w.B, w.T, HN)[torch.as_tensor(sb, device=device), :, torch.as_tensor(shn, device=device)]
+        return float(np.max(np.abs(got.T.double().cpu().numpy() - ref) / ref))
+
+    err_lti = lam_err(outs[0])
+    # the general scan on the same problem
+    a_full = d["a"][:, None].expand(w.B, w.T, w.H, w.N).contiguous()
+    p_full = torch.zeros_like(a_full)
+    gws = kla.new_workspace(w.B, w.T, w.H, w.N, torch.float32, device)
+    gargs = (a_full, p_full, d["phi"], d["b"], d["lam0"], d["eta0"])
+    gper = time_launches(lambda: kla.scan_forward(*gargs, out=outs, workspace=gws), steps, warmup)
+    gms = statistics.median(gper)
+    err_gen = lam_err(outs[0])
+    del a_full, p_full, gws, d, outs, ws
+    return {"workload": w.summary, "ms": ms, "value": tc / (ms * 1e-3), "unit": UNIT, "gb_per_s": gbs,
+            "launches_timed": steps,
+            "kernel": {1: "kla_lti_seq_kernel (one thread per channel)",
+                       2: "kla_lti_stream_kernel (channel-owning streaming, blocked convolutions)"}[plan[0]],
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "algorithmic_bytes_per_launch": bpt * tc, "bytes_per_token_channel": bpt},
+            "max_rel_err_lambda_vs_oracle": err_lti,
+            "general_scan_same_problem": {
+                "ms": gms, "value": tc / (gms * 1e-3), "bytes_per_token_channel": 32,
+                "gb_per_s": 32 * tc / (gms * 1e-3) / 1e9, "max_rel_err_lambda_vs_oracle": err_gen,
+                "speedup_of_convolutional_form": gms / ms},
+            "timing": "median of per-launch CUDA events (inputs of 2.1 GB, larger than L2)"}
+
+
+def time_attention(kla, device, steps: int, warmup: int, peak: float, W: int = 64):
+    """kla_attention_weights over every window of W tokens of the LM-layer
+    workload (bf16 inputs), from the forward scan's lambda."""
+    import torch
+    w = wl.WORKLOADS["lm_layer"]
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(x[k]).to(device=device, dtype=torch.bfloat16) for k in wl.INPUT_NAMES}
+    lam0 = torch.from_numpy(x["lam0"]).to(device)
+    eta0 = torch.from_numpy(x["eta0"]).to(device)
+    del x
+    lam = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], lam0, eta0, want_mu=False, want_var=False)[0]
+    del d["phi"], d["b"]
+    nwin = -(-w.T // W)
+    F = torch.empty((w.B, nwin, W, W, w.H, w.N), device=device)
+    per = time_launches(lambda: kla.attention_weights(d["a"], d["p"], lam, W=W, out=F), steps, warmup)
+    if kla.get_error() != 0:
+        raise RuntimeError("device-side error in the attention weights")
+    ms = statistics.median(per)
+    HN = w.H * w.N
+    write_bytes = w.B * nwin * W * W * HN * 4
+    read_bytes = w.token_channels * (2 + 2 + 4)
+    gbs = (write_bytes + read_bytes) / (ms * 1e-3) / 1e9
+    del F, lam, d
+    return {"workload": f"Kalman attention weights, windows of {W} tokens over {w.summary}", "ms": ms,
+            "value": w.token_channels / (ms * 1e-3), "unit": UNIT, "gb_per_s": gbs, "launches_timed": steps,
+            "kernel": "kla_attention_kernel", "weights_per_s": write_bytes / 4 / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "algorithmic_bytes_per_launch": write_bytes + read_bytes,
+                         "bytes": f"{W}*{W}*4 written per channel and window + a, p (bf16) and lambda read"},
+            "timing": "median of per-launch CUDA events (8.6 GB written per launch, larger than L2)"}
+
+
 def backward_bytes_per_tc(w: wl.Workload) -> int:
     """Bytes the backward scan must move per token-channel with all four
     output gradients present: read a, p (input dtype), lambda, eta and the
@@ -667,6 +758,15 @@ def run_ours(args):
                 configs[name]["cpu_baseline_1core"] = cpu_oracle_sample(w_c, host_cfg[name], args.cpu_target_s,
                                                                         threads=1)
         del host_cfg
+        if not args.no_forms:
+            torch.cuda.empty_cache()
+            configs["lti"] = time_lti(kla, device, args.config_steps, args.warmup, peak)
+            torch.cuda.empty_cache()
+            configs["attention"] = time_attention(kla, device, args.config_steps, args.warmup, peak)
+            torch.cuda.empty_cache()
+            for name in ("lti", "attention"):
+                configs[name]["roofline"]["frac_of_same_run_copy"] = (configs[name]["gb_per_s"]
+                                                                      / copy_bw["gb_per_s"])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and host is not None:
@@ -767,6 +867,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-configs", action="store_true",
                     help="skip timing the tiny, LM-layer and stiff workloads on their own")
     ap.add_argument("--config-steps", type=int, default=30)
+    ap.add_argument("--no-forms", action="store_true",
+                    help="skip the convolutional-form and attention-weight legs")
     ap.add_argument("--cpu-target-s", type=float, default=4.0,
                     help="seconds of oracle work per CPU timing of the per-workload entries")
     return ap.parse_args(argv)

@@ -399,6 +399,95 @@ kla_status_t kla_layer_step(const void *k, const void *q, const void *v, const v
                             const float *a, const float *p, float *lambda_state, float *eta_state,
                             float *y, float *s, int64_t B, int64_t H, int64_t D, int64_t Ns, void *stream);
 
+/* Largest window (tokens) of kla_attention_weights. */
+#define KLA_ATTENTION_MAX_WINDOW 64
+
+/*
+ * The Kalman attention weights: how the information mean of a later token
+ * responds to an earlier one (the review's "Kalman Attention Matrix", its
+ * minor comment on App. E.3/E.4).  The affine recursion eta_k = f_k eta_{k-1}
+ * + b_k (review "Core claim") unrolls into
+ *
+ *   eta_t = F(t, s) eta_s + sum_{r = s+1..t} F(t, r) b_r,
+ *   F(t, s) = prod_{k = s+1..t} f_k,   f_k = a_k / (a_k^2 + p_k lambda_{k-1}),
+ *
+ * (rows 0-based; F(t, t) = 1), which also equals prod(a) / (C lambda_s + D)
+ * for [[A, B], [C, D]] = M_t ... M_{s+1}.  The tokens [t0, t0 + span) are cut
+ * into windows of W tokens and F is written for every pair inside a window:
+ *
+ *   a, p        [B, T, H, N] forward inputs, dtype in_dtype (read only)
+ *   lambda_out  [B, T, H, N] fp32 posterior precision written by
+ *               kla_scan_forward on the same inputs (read only; the gate of
+ *               token k uses row k-1)
+ *   F           [B, nwin, W, W, H, N] fp32, nwin = ceil(span / W) (written):
+ *               F[b, w, i, j, h, n] = F(t, s) with t = t0 + w W + i,
+ *               s = t0 + w W + j, for j <= i < (tokens of window w inside the
+ *               span); every other entry (above the diagonal, past the span)
+ *               is written as 0.
+ *
+ * 1 <= W <= KLA_ATTENTION_MAX_WINDOW and 0 <= t0 <= t0 + span <= T, else
+ * KLA_ERR_INVALID_ARG.  span == 0 or B*H*N == 0 is a valid empty call.  F may
+ * not overlap the inputs.  The gates use the hardware reciprocal, as the
+ * scan does; the products are plain fp32 multiplies (an entry below the fp32
+ * normal range flushes to 0).  Bound by the bytes of F: W^2 * 4 per channel
+ * and window.
+ */
+kla_status_t kla_attention_weights(const void *a, const void *p, kla_dtype_t in_dtype,
+                                   const float *lambda_out, float *F,
+                                   int64_t B, int64_t T, int64_t H, int64_t N,
+                                   int64_t t0, int64_t span, int64_t W, void *stream);
+
+/*
+ * Device workspace that kla_scan_forward_lti needs (run-boundary carries and
+ * flags), written to *bytes; 0 for an empty problem.
+ */
+kla_status_t kla_scan_forward_lti_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                                 kla_dtype_t in_dtype, size_t *bytes);
+
+/*
+ * The filter of deterministic time-invariant channels in its convolutional
+ * form (the review's Theorem 3: for a deterministic LTI system the filter is
+ * a convolution).  With no process noise (p_t = 0) and a decay a constant in
+ * time, the precision map is affine and the gate is 1/a, so (rows 0-based)
+ *
+ *   lambda_t = a^(-2(t+1)) lambda_0 + sum_{s<=t} a^(-2(t-s)) phi_s,
+ *   eta_t    = a^(-(t+1))  eta_0    + sum_{s<=t} a^(-(t-s))  b_s,
+ *
+ * mu_t = eta_t / lambda_t, var_t = 1 / lambda_t: the same results as
+ * kla_scan_forward with a_t = a and p_t = 0, computed as blocked causal
+ * convolutions with the geometric kernels and reading only phi and b per
+ * token.  The carry between chunks is kept in fp64, so a constant decay does
+ * not accumulate a drift over long sequences.
+ *
+ *   a              [B, H, N] fp32 decay of each channel, nonzero (read only)
+ *   phi, b         [B, T, H, N] dtype in_dtype (read only)
+ *   lambda0, eta0  [B, H, N] fp32 prior (read only)
+ *   lambda_out, eta_out, mu_out, var_out
+ *                  [B, T, H, N] fp32 outputs, as for kla_scan_forward (mu_out
+ *                  and var_out may be NULL)
+ *   workspace      at least kla_scan_forward_lti_workspace_size(...) bytes,
+ *                  256-byte aligned; contents on entry do not matter
+ *
+ * Preconditions as for kla_scan_forward; the state must stay in fp32 range
+ * (with |a| < 1 the precision grows like a^(-2t)).  Empty problems are valid.
+ */
+kla_status_t kla_scan_forward_lti(const float *a, const void *phi, const void *b, kla_dtype_t in_dtype,
+                                  const float *lambda0, const float *eta0,
+                                  float *lambda_out, float *eta_out, float *mu_out, float *var_out,
+                                  int64_t B, int64_t T, int64_t H, int64_t N,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Which kernel kla_scan_forward_lti would launch (only the alignment of phi
+ * and b is looked at), written to *kernel: 1 = one thread per channel (any
+ * shape), 2 = the channel-owning streaming kernel (16-byte aligned arrays,
+ * H*N*elem a multiple of 16 bytes, H*N >= 32, T >= 32); *launches = kernel
+ * launches per call (2 when a workspace clear precedes the streaming
+ * kernel).  0 and 0 for an empty problem.
+ */
+kla_status_t kla_scan_forward_lti_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
+                                       const void *phi, const void *b, int *kernel, int *launches);
+
 /*
  * Synchronise `stream`, then report the first failure since the previous
  * call on the current device: KLA_ERR_CUDA for a CUDA error (sticky or not),

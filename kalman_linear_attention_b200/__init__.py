@@ -13,6 +13,7 @@ _API_NAMES = {
     "KlaError", "lib", "load_library", "scan_forward_static",
     "scan_backward", "backward_workspace_size", "backward_plan", "debug_force_backward_kernel",
     "KalmanFilterScan", "kalman_filter", "layer_forward", "layer_workspace_size", "layer_step",
+    "attention_weights", "scan_forward_lti", "lti_workspace_size", "lti_plan",
 }
 
 

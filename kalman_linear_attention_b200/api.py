@@ -64,7 +64,16 @@ SIGNATURES = {
                                          _VP, _I64, _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
     "kla_layer_step": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP,
                                       _I64, _I64, _I64, _I64, _VP]),
+    "kla_attention_weights": (ctypes.c_int, [_VP, _VP, ctypes.c_int, _VP, _VP, _I64, _I64, _I64, _I64,
+                                             _I64, _I64, _I64, _VP]),
+    "kla_scan_forward_lti_workspace_size": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int,
+                                                           ctypes.POINTER(_SZ)]),
+    "kla_scan_forward_lti": (ctypes.c_int, [_VP, _VP, _VP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _VP,
+                                            _I64, _I64, _I64, _I64, _VP, _SZ, _VP]),
+    "kla_scan_forward_lti_plan": (ctypes.c_int, [_I64, _I64, _I64, _I64, ctypes.c_int, _VP, _VP,
+                                                 ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
 }
+ATTENTION_MAX_WINDOW = 64  # KLA_ATTENTION_MAX_WINDOW
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -509,3 +518,85 @@ def layer_step(k: torch.Tensor, q: torch.Tensor, v: torch.Tensor, w: torch.Tenso
                                   _stream_handle(stream))
     _check(st, "kla_layer_step")
     return y, s
+
+
+def attention_weights(a: torch.Tensor, p: torch.Tensor, lam: torch.Tensor, *, t0: int = 0,
+                      span: Optional[int] = None, W: int = ATTENTION_MAX_WINDOW,
+                      out: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The Kalman attention weights F(t, s) = prod_{k=s+1..t} f_k of the
+    windows of W tokens of [t0, t0 + span), from the forward inputs a, p and
+    the forward scan's lambda ([B, T, H, N]).  Returns fp32
+    [B, ceil(span / W), W, W, H, N] (kla_attention_weights)."""
+    if a.dim() != 4 or p.shape != a.shape or lam.shape != a.shape:
+        raise ValueError("a, p, lam must share one [B, T, H, N] shape")
+    if p.dtype != a.dtype or lam.dtype != torch.float32:
+        raise TypeError("a and p share one dtype; lam is float32")
+    B, T, H, N = a.shape
+    span = T - t0 if span is None else span
+    nwin = -(-span // W) if W > 0 else 0
+    _require_cuda(a, p, lam)
+    if out is None:
+        out = torch.empty((B, nwin, W, W, H, N), dtype=torch.float32, device=a.device)
+    else:
+        _require_cuda(out)
+        if out.shape != (B, nwin, W, W, H, N) or out.dtype != torch.float32:
+            raise ValueError("out must be float32 [B, nwin, W, W, H, N]")
+    with torch.cuda.device(a.device):
+        _check(lib().kla_attention_weights(_ptr(a), _ptr(p), _dtype_code(a), _ptr(lam), _ptr(out), B, T, H, N,
+                                           t0, span, W, _stream_handle(stream)), "kla_attention_weights")
+    return out
+
+
+def lti_workspace_size(B: int, T: int, H: int, N: int, dtype: torch.dtype = torch.float32) -> int:
+    code = KLA_BF16 if dtype == torch.bfloat16 else KLA_F32
+    out = ctypes.c_size_t(0)
+    _check(lib().kla_scan_forward_lti_workspace_size(B, T, H, N, code, ctypes.byref(out)),
+           "kla_scan_forward_lti_workspace_size")
+    return int(out.value)
+
+
+def lti_plan(phi: torch.Tensor, b: torch.Tensor) -> Tuple[int, int]:
+    """(kernel, launches) of scan_forward_lti: 1 = one thread per channel,
+    2 = channel-owning streaming."""
+    B, T, H, N = phi.shape
+    k, n = ctypes.c_int(0), ctypes.c_int(0)
+    with torch.cuda.device(phi.device):
+        _check(lib().kla_scan_forward_lti_plan(B, T, H, N, _dtype_code(phi), _ptr(phi), _ptr(b), ctypes.byref(k),
+                                               ctypes.byref(n)), "kla_scan_forward_lti_plan")
+    return int(k.value), int(n.value)
+
+
+def scan_forward_lti(a: torch.Tensor, phi: torch.Tensor, b: torch.Tensor, lam0: torch.Tensor,
+                     eta0: torch.Tensor, *, want_mu: bool = True, want_var: bool = True,
+                     out: Optional[Sequence[Optional[torch.Tensor]]] = None,
+                     workspace: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None,
+                     ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
+    """The deterministic time-invariant filter (p = 0, decay a [B, H, N]
+    constant in time) in its convolutional form (kla_scan_forward_lti):
+    phi, b [B, T, H, N]; returns (lambda, eta, mu, var) as scan_forward does."""
+    if phi.dim() != 4 or b.shape != phi.shape or b.dtype != phi.dtype:
+        raise ValueError("phi, b must share one [B, T, H, N] shape and dtype")
+    B, T, H, N = phi.shape
+    for t, name in ((a, "a"), (lam0, "lam0"), (eta0, "eta0")):
+        if t.shape != (B, H, N) or t.dtype != torch.float32:
+            raise ValueError(f"{name} must be float32 [B, H, N]")
+    _require_cuda(a, phi, b, lam0, eta0)
+    dev = phi.device
+    if out is None:
+        outs = [torch.empty((B, T, H, N), dtype=torch.float32, device=dev),
+                torch.empty((B, T, H, N), dtype=torch.float32, device=dev),
+                torch.empty((B, T, H, N), dtype=torch.float32, device=dev) if want_mu else None,
+                torch.empty((B, T, H, N), dtype=torch.float32, device=dev) if want_var else None]
+    else:
+        outs = list(out)
+        _require_cuda(*[o for o in outs if o is not None])
+    if workspace is None:
+        workspace = torch.empty(max(lti_workspace_size(B, T, H, N, phi.dtype), 1), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().kla_scan_forward_lti(_ptr(a), _ptr(phi), _ptr(b), _dtype_code(phi), _ptr(lam0), _ptr(eta0),
+                                        _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), B, T, H, N,
+                                        _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(st, "kla_scan_forward_lti")
+    return tuple(outs)

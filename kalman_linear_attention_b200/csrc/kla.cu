@@ -19,7 +19,9 @@
 #include "kla_backward.cuh"
 #include "kla_forward.cuh"
 #include "kla_forward_stream.cuh"
+#include "kla_attention.cuh"
 #include "kla_layer.cuh"
+#include "kla_lti.cuh"
 #include "kla_step.cuh"
 
 #define KLA_API extern "C" __attribute__((visibility("default")))
@@ -1096,4 +1098,220 @@ KLA_API kla_status_t kla_layer_step(const void *k, const void *q, const void *v,
         e = Ns == 8 ? cudaLaunchKernelEx(&cfg, kla::kla_layer_step_kernel<__nv_bfloat16, 8>, prm)
                     : cudaLaunchKernelEx(&cfg, kla::kla_layer_step_kernel<__nv_bfloat16, 16>, prm);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// The Kalman attention weights: kla_attention_weights (kernel in
+// kla_attention.cuh).
+// ---------------------------------------------------------------------------
+KLA_API kla_status_t kla_attention_weights(const void *a, const void *p, kla_dtype_t in_dtype,
+                                           const float *lambda_out, float *F, int64_t B, int64_t T,
+                                           int64_t H, int64_t N, int64_t t0, int64_t span, int64_t W,
+                                           void *stream) {
+    if (B < 0 || T < 0 || H < 0 || N < 0 || t0 < 0 || span < 0) return KLA_ERR_INVALID_ARG;
+    if (W < 1 || W > KLA_ATTENTION_MAX_WINDOW) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    if (t0 > T || span > T - t0) return KLA_ERR_INVALID_ARG;
+    int64_t HN = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems)) return KLA_ERR_INVALID_ARG;
+    if (span == 0 || B == 0 || HN == 0) return KLA_OK;
+    if (!a || !p || !lambda_out || !F) return KLA_ERR_INVALID_ARG;
+    const int64_t nwin = (span + W - 1) / W;
+    int64_t bw = 0, bww = 0, f_elems = 0, f_bytes = 0, in_bytes = 0, l_bytes = 0;
+    if (!mul_ok(B, nwin, &bw) || !mul_ok(bw, W * W, &bww) || !mul_ok(bww, HN, &f_elems) ||
+        !mul_ok(f_elems, 4, &f_bytes) || !mul_ok(elems, (int64_t)dtype_size(in_dtype), &in_bytes) ||
+        !mul_ok(elems, 4, &l_bytes))
+        return KLA_ERR_INVALID_ARG;
+    const Range outs[1] = {range_of(F, f_bytes)};
+    const Range ins[3] = {range_of(a, in_bytes), range_of(p, in_bytes), range_of(lambda_out, l_bytes)};
+    if (any_overlap(outs, 1, ins, 3)) return KLA_ERR_INVALID_ARG;
+    const bool vec4 = HN % 4 == 0 && aligned16(F);
+    const int cw = vec4 ? 128 : 32;
+    const int64_t nct = (HN + cw - 1) / cw;
+    int64_t grid = 0;
+    if (!mul_ok(bw, nct, &grid) || grid > kMaxGrid || nwin > INT32_MAX) return KLA_ERR_INVALID_ARG;
+    kla::AttnParams prm;
+    prm.a = a; prm.p = p; prm.lam = lambda_out; prm.F = F;
+    prm.T = T; prm.HN = HN; prm.t0 = t0; prm.span = span;
+    prm.W = (int)W; prm.nwin = (int)nwin; prm.nct = nct;
+    const size_t smem = (size_t)W * cw * sizeof(float);  // <= 32 KB
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (in_dtype == KLA_F32) {
+        if (vec4) kla::kla_attention_kernel<float, 4><<<(unsigned)grid, 256, smem, st>>>(prm);
+        else kla::kla_attention_kernel<float, 1><<<(unsigned)grid, 256, smem, st>>>(prm);
+    } else {
+        if (vec4) kla::kla_attention_kernel<__nv_bfloat16, 4><<<(unsigned)grid, 256, smem, st>>>(prm);
+        else kla::kla_attention_kernel<__nv_bfloat16, 1><<<(unsigned)grid, 256, smem, st>>>(prm);
+    }
+    return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// The convolutional form of deterministic time-invariant channels:
+// kla_scan_forward_lti (kernels in kla_lti.cuh).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Chunk warps of the convolutional-form kernel (the chunk in registers is
+// half the general scan's: phi and b only) and tokens per sub-block of its
+// local convolutions.
+#ifndef KLA_LTI_W
+#define KLA_LTI_W 8
+#endif
+#ifndef KLA_LTI_S
+#define KLA_LTI_S 8
+#endif
+constexpr int kLtiL = 32;
+constexpr int kLtiG = 8;
+
+template <typename Tin>
+constexpr int lti_stages() {
+    constexpr int W = KLA_LTI_W;
+    const int stage = 2 * kLtiL * 32 * (int)sizeof(Tin);
+    const int fixed = W * 2 * 4 * kLtiG * 32 * 4 + W * 2 * 32 * 8 + W * 8 + 2048;
+    const int ns = (KLA_STREAM_SMEM - fixed) / stage;
+    return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
+}
+
+template <typename Tin>
+cudaError_t launch_lti_stream(const kla::LtiParams &prm, const kla::LtiMaps &maps, cudaStream_t stream) {
+    constexpr int NS = lti_stages<Tin>();
+    using Cfg = kla::LtiTile<Tin, kLtiL, KLA_LTI_W, NS, kLtiG>;
+    static_assert(NS >= KLA_LTI_W && Cfg::SMEM <= 227 * 1024, "convolutional-form kernel shared memory");
+    auto kernel = kla::kla_lti_stream_kernel<Tin, kLtiL, KLA_LTI_S, KLA_LTI_W, NS, kLtiG>;
+    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
+    kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    return cudaGetLastError();
+}
+
+// Run-split workspace of the convolutional form: ticket, one flag per run
+// boundary, fp64 (lambda, eta) of 32 channels per boundary.
+StreamWs lti_ws_layout(int64_t ntiles, int parts) {
+    StreamWs w;
+    const size_t nb = (size_t)ntiles * (size_t)(parts - 1);
+    w.flags_off = kHeaderBytes;
+    w.state_off = w.flags_off + round_up(nb * sizeof(unsigned), 256);
+    w.clear_bytes = w.state_off;
+    w.total = w.state_off + round_up(nb * 64 * sizeof(double), 256);
+    return w;
+}
+
+// 2: the streaming kernel (TMA geometry as for the general streaming scan:
+// 16-byte aligned phi, b and outputs, H*N*elem a multiple of 16 bytes,
+// H*N >= 32, T >= 32); 1: one thread per channel (any shape).
+int lti_kernel_choice(int64_t T, int64_t HN, size_t esz, const void *const *ptrs, int n) {
+    bool ok = (HN * (int64_t)esz) % 16 == 0 && T >= kLtiL && HN >= 32 && encode_fn() != nullptr;
+    for (int k = 0; k < n && ok; ++k)
+        if (ptrs[k] && !aligned16(ptrs[k])) ok = false;
+    return ok ? 2 : 1;
+}
+
+}  // namespace
+
+KLA_API kla_status_t kla_scan_forward_lti_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
+                                                         kla_dtype_t in_dtype, size_t *bytes) {
+    if (!bytes || B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems)) return KLA_ERR_INVALID_ARG;
+    *bytes = elems == 0 ? 0 : lti_ws_layout(B * ((HN + 31) / 32), KLA_STREAM_MAX_PARTS).total;
+    return KLA_OK;
+}
+
+KLA_API kla_status_t kla_scan_forward_lti(const float *a, const void *phi, const void *b, kla_dtype_t in_dtype,
+                                          const float *lambda0, const float *eta0, float *lambda_out,
+                                          float *eta_out, float *mu_out, float *var_out, int64_t B, int64_t T,
+                                          int64_t H, int64_t N, void *workspace, size_t workspace_bytes,
+                                          void *stream) {
+    if (B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, C = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, HN, &C) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems))
+        return KLA_ERR_INVALID_ARG;
+    if (elems == 0) return KLA_OK;
+    if (!a || !phi || !b || !lambda0 || !eta0 || !lambda_out || !eta_out) return KLA_ERR_INVALID_ARG;
+    const size_t esz = dtype_size(in_dtype);
+    int64_t in_bytes = 0, out_bytes = 0;
+    if (!mul_ok(elems, (int64_t)esz, &in_bytes) || !mul_ok(elems, 4, &out_bytes)) return KLA_ERR_INVALID_ARG;
+    const Range outs[5] = {range_of(lambda_out, out_bytes), range_of(eta_out, out_bytes),
+                           range_of(mu_out, out_bytes), range_of(var_out, out_bytes),
+                           range_of(workspace, (int64_t)workspace_bytes)};
+    const Range ins[5] = {range_of(a, C * 4), range_of(phi, in_bytes), range_of(b, in_bytes),
+                          range_of(lambda0, C * 4), range_of(eta0, C * 4)};
+    if (any_overlap(outs, 5, ins, 5)) return KLA_ERR_INVALID_ARG;
+    size_t need = 0;
+    if (kla_scan_forward_lti_workspace_size(B, T, H, N, in_dtype, &need) != KLA_OK) return KLA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need) return KLA_ERR_WORKSPACE_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KLA_ERR_MISALIGNED;
+    if (T > INT32_MAX - 64 || HN > INT32_MAX || B > INT32_MAX) return KLA_ERR_INVALID_ARG;
+
+    kla::LtiParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.a = a; prm.lam0 = lambda0; prm.eta0 = eta0;
+    prm.T = T; prm.HN = HN;
+    prm.write_mu = mu_out != nullptr; prm.write_var = var_out != nullptr;
+    prm.wait_ns = g_wait_ns.load();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const void *ptrs[6] = {phi, b, lambda_out, eta_out, mu_out, var_out};
+    if (lti_kernel_choice(T, HN, esz, ptrs, 6) == 2) {
+        const CUtensorMapDataType tdt =
+            in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        kla::LtiMaps maps;
+        std::memset(&maps, 0, sizeof(maps));
+        bool ok = encode_stream_map(&maps.in[0], phi, tdt, esz, B, T, HN, kLtiL) &&
+                  encode_stream_map(&maps.in[1], b, tdt, esz, B, T, HN, kLtiL);
+        float *outs4[4] = {lambda_out, eta_out, mu_out, var_out};
+        for (int k = 0; k < 4 && ok; ++k)
+            if (outs4[k]) ok = encode_stream_map(&maps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T,
+                                                 HN, kLtiG);
+        if (ok) {
+            prm.ntiles = B * ((HN + 31) / 32);
+            prm.nct = (int)((HN + 31) / 32);
+            prm.nchunks = (int)((T + kLtiL - 1) / kLtiL);
+            prm.parts = stream_parts(prm.ntiles, prm.nchunks);
+            prm.chunks_per_part = (prm.nchunks + prm.parts - 1) / prm.parts;
+            prm.nunits = prm.ntiles * prm.parts;
+            unsigned char *ws = static_cast<unsigned char *>(workspace);
+            prm.ticket = reinterpret_cast<unsigned *>(ws);
+            if (prm.parts > 1) {
+                const StreamWs sw = lti_ws_layout(prm.ntiles, prm.parts);
+                if (sw.total > workspace_bytes) return KLA_ERR_WORKSPACE_TOO_SMALL;
+                prm.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
+                prm.part_state = reinterpret_cast<double *>(ws + sw.state_off);
+                if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
+            }
+            const cudaError_t e = in_dtype == KLA_F32 ? launch_lti_stream<float>(prm, maps, st)
+                                                      : launch_lti_stream<__nv_bfloat16>(prm, maps, st);
+            return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+        }
+    }
+    const int threads = 128;
+    const int64_t blocks = (C + threads - 1) / threads;
+    if (in_dtype == KLA_F32)
+        kla::kla_lti_seq_kernel<float, KLA_LTI_S><<<(unsigned)blocks, threads, 0, st>>>(
+            prm, phi, b, lambda_out, eta_out, mu_out, var_out, C);
+    else
+        kla::kla_lti_seq_kernel<__nv_bfloat16, KLA_LTI_S><<<(unsigned)blocks, threads, 0, st>>>(
+            prm, phi, b, lambda_out, eta_out, mu_out, var_out, C);
+    return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+KLA_API kla_status_t kla_scan_forward_lti_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
+                                               const void *phi, const void *b, int *kernel, int *launches) {
+    if (!kernel || !launches || B < 0 || T < 0 || H < 0 || N < 0) return KLA_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return KLA_ERR_UNSUPPORTED_DTYPE;
+    int64_t HN = 0, BT = 0, elems = 0;
+    if (!mul_ok(H, N, &HN) || !mul_ok(B, T, &BT) || !mul_ok(BT, HN, &elems)) return KLA_ERR_INVALID_ARG;
+    if (elems == 0) {
+        *kernel = 0;
+        *launches = 0;
+        return KLA_OK;
+    }
+    const void *ptrs[2] = {phi, b};
+    *kernel = lti_kernel_choice(T, HN, dtype_size(in_dtype), ptrs, 2);
+    *launches = 1;
+    if (*kernel == 2 && stream_parts(B * ((HN + 31) / 32), (T + kLtiL - 1) / kLtiL) > 1) *launches = 2;
+    return KLA_OK;
 }

@@ -1,0 +1,123 @@
+// kla_attention.cuh -- the Kalman attention weights of the information mean
+// (sm_100a).
+//
+// Between two tokens s <= t of one channel the information mean of the later
+// token responds to the earlier one through the gates between them: the
+// affine recursion eta_k = f_k eta_{k-1} + b_k (KLA review, "Core claim")
+// unrolls into
+//
+//   eta_t = F(t, s) eta_s + sum_{r = s+1..t} F(t, r) b_r,
+//   F(t, s) = prod_{k = s+1..t} f_k,   f_k = a_k / (a_k^2 + p_k lambda_{k-1}),
+//
+// a lower-triangular matrix of weights per channel -- the review's "Kalman
+// Attention Matrix" (minor comment on its App. E.3/E.4).  By the telescoping
+// denominators of the Moebius product it also equals prod(a) / (C lambda_s +
+// D) with [[A, B], [C, D]] = M_t ... M_{s+1}.
+//
+// One CTA owns one window of W tokens of one batch row and a tile of 32 x VEC
+// channels.  Its threads first form the window's gates from a, p and the
+// forward scan's stored lambda (one reciprocal per token and channel, into
+// shared memory); then each warp writes whole columns s of the W x W matrix,
+// lane = VEC channels: the running product down the column is one multiply
+// per entry, and every entry, the zeros above the diagonal included, leaves
+// with one streaming store of 16 bytes (VEC = 4) per lane.  Output traffic
+// (W^2 floats per channel and window) dominates: the kernel is bound by HBM
+// writes.
+#pragma once
+
+#include "kla_device.cuh"
+
+namespace kla {
+
+struct AttnParams {
+    const void *a, *p;             // [B, T, H, N], input dtype
+    const float *lam;              // [B, T, H, N] posterior precision of the forward scan
+    float *F;                      // [B, nwin, W, W, H, N]
+    int64_t T, HN;
+    int64_t t0, span;              // tokens [t0, t0 + span), cut into windows of W
+    int W, nwin;
+    int64_t nct;                   // channel tiles (of 32 x VEC) per batch row
+};
+
+// VEC consecutive floats: streaming (evict-first) global store, shared load.
+__device__ __forceinline__ void st_cs_vec(float *dst, const float (&v)[1]) { __stcs(dst, v[0]); }
+__device__ __forceinline__ void st_cs_vec(float *dst, const float (&v)[4]) {
+    __stcs(reinterpret_cast<float4 *>(dst), make_float4(v[0], v[1], v[2], v[3]));
+}
+__device__ __forceinline__ void lds_vec(float (&v)[1], const float *src) { v[0] = *src; }
+__device__ __forceinline__ void lds_vec(float (&v)[4], const float *src) {
+    const float4 x = *reinterpret_cast<const float4 *>(src);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+
+// Grid: one CTA per (batch row, window, channel tile), flattened on x as
+// ((b * nwin) + window) * nct + tile.  Dynamic shared memory: W * 32 * VEC
+// floats of gates.
+template <typename Tin, int VEC>
+__global__ void __launch_bounds__(256) kla_attention_kernel(const AttnParams prm) {
+    constexpr int CW = 32 * VEC;
+    extern __shared__ __align__(16) float gates[];  // [W][CW]
+    const int64_t cta = blockIdx.x;
+    const int64_t tile = cta % prm.nct;
+    const int64_t bw = cta / prm.nct;
+    const int win = (int)(bw % prm.nwin);
+    const int64_t bb = bw / prm.nwin;
+    const int64_t start = prm.t0 + (int64_t)win * prm.W;
+    const int64_t left = prm.t0 + prm.span - start;
+    const int nv = (int)(left < (int64_t)prm.W ? left : (int64_t)prm.W);  // tokens of this window in the span
+    const int64_t c0 = tile * CW;
+    const Tin *ag = static_cast<const Tin *>(prm.a);
+    const Tin *pg = static_cast<const Tin *>(prm.p);
+
+    // 1) the gate of every window token after the first (the first one's is
+    //    never used: F(t, s) takes the gates of tokens s+1..t)
+    for (int idx = threadIdx.x; idx < nv * CW; idx += blockDim.x) {
+        const int k = idx / CW;
+        const int c = idx - k * CW;
+        float g = 0.f;
+        if (k >= 1 && c0 + c < prm.HN) {
+            const int64_t row = (bb * prm.T + start + k) * prm.HN + c0 + c;
+            const float a = to_f32(ag[row]);
+            const float p = to_f32(pg[row]);
+            const float lam_before = __ldg(prm.lam + row - prm.HN);  // lambda_{k-1}: this channel, previous token
+            g = a * rcp_hw(fmaf(p, lam_before, a * a));
+        }
+        gates[idx] = g;
+    }
+    __syncthreads();
+
+    // 2) columns: warp w writes columns w, w + nwarps, ...; every column holds
+    //    W entries, so the stores are balanced across warps
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const bool cvalid = c0 + lane * VEC < prm.HN;  // VEC = 4 needs H*N % 4 == 0: whole vectors
+    const int64_t WW = (int64_t)prm.W * prm.W;
+    float *Fcta = prm.F + ((bb * prm.nwin + win) * WW) * prm.HN + c0 + lane * VEC;
+    const float *glane = gates + lane * VEC;
+#pragma unroll 1
+    for (int j = warp; j < prm.W; j += nwarps) {
+        float f[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) f[v] = 1.f;
+        float *col = Fcta + (int64_t)j * prm.HN;
+        const float zero[VEC] = {};
+#pragma unroll 1
+        for (int i = 0; i < prm.W; ++i) {
+            float *dst = col + (int64_t)i * prm.W * prm.HN;
+            if (i < j || i >= nv || j >= nv) {
+                if (cvalid) st_cs_vec(dst, zero);
+            } else {
+                if (i > j) {
+                    float g[VEC];
+                    lds_vec(g, glane + i * CW);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) f[v] *= g[v];
+                }
+                if (cvalid) st_cs_vec(dst, f);
+            }
+        }
+    }
+}
+
+}  // namespace kla

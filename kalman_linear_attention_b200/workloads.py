@@ -320,6 +320,64 @@ def random_layer_prior(w: LayerWorkload, seed: int = 778) -> Dict[str, np.ndarra
             "eta0": rng.standard_normal(shape).astype(np.float32)}
 
 
+# --------------------------------------------------------------------------
+# Deterministic time-invariant channels (the convolutional form): p = 0 and a
+# decay per channel, constant in time.  phi and b are the "base" family's
+# streams of the same seed (drawn exactly as for a ``base`` workload); a is
+# drawn per channel from its own stream, U(a_lo, a_hi) fp32 [B, H, N].
+LTI_WORKLOADS: Dict[str, Workload] = {
+    "lti": Workload("lti", 1, 32, 128, 65536, "f32", "base", 6,
+                    summary="deterministic time-invariant forward scan (convolutional form), fp32, "
+                            "B=1 H=32 N=128 T=65536, p=0, a~U(0.9995,1.0005) per channel"),
+}
+LTI_DECAY_RANGE = (0.9995, 1.0005)
+
+
+def iter_lti_rows(w: Workload, rows_per_block: int | None = None
+                  ) -> Iterator[Tuple[int, int, Dict[str, np.ndarray]]]:
+    """Like iter_rows, for phi and b only (fp32 [rows, H, N] blocks)."""
+    HN = w.H * w.N
+    rows = w.B * w.T
+    if rows_per_block is None:
+        rows_per_block = max(1, _BLOCK_ELEMS // max(HN, 1))
+    rngs = _streams(w.seed)[2:]
+
+    def one(name, rng, n):
+        x = _draw(w.dist, name, rng, n).astype(np.float32)
+        return round_to_bf16(x) if w.dtype == "bf16" else x
+
+    with ThreadPoolExecutor(max_workers=2) as pool:
+        r0 = 0
+        while r0 < rows:
+            r1 = min(rows, r0 + rows_per_block)
+            n = (r1 - r0) * HN
+            futs = [pool.submit(one, name, rng, n) for name, rng in zip(("phi", "b"), rngs)]
+            yield r0, r1, {name: f.result().reshape(r1 - r0, w.H, w.N) for name, f in zip(("phi", "b"), futs)}
+            r0 = r1
+
+
+def lti_decay(w: Workload, lo: float = LTI_DECAY_RANGE[0], hi: float = LTI_DECAY_RANGE[1]) -> np.ndarray:
+    """The per-channel decay of a time-invariant workload: U(lo, hi), fp32 [B, H, N]."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, 3])))
+    return rng.uniform(lo, hi, (w.B, w.H, w.N)).astype(np.float32)
+
+
+def generate_lti(w: Workload, decay: Tuple[float, float] = LTI_DECAY_RANGE) -> Dict[str, np.ndarray]:
+    """All inputs of a time-invariant workload: a [B, H, N], phi, b
+    [B, T, H, N] (fp32 arrays; bf16-rounded values for bf16 workloads),
+    lam0 = 1, eta0 = 0 [B, H, N]."""
+    HN = w.H * w.N
+    full = {k: np.empty((w.B * w.T, w.H, w.N), dtype=np.float32) for k in ("phi", "b")}
+    if w.B * w.T * HN:
+        for r0, r1, blk in iter_lti_rows(w):
+            for k in ("phi", "b"):
+                full[k][r0:r1] = blk[k]
+    out = {k: v.reshape(w.B, w.T, w.H, w.N) for k, v in full.items()}
+    out["a"] = lti_decay(w, *decay)
+    out.update(prior(w))
+    return out
+
+
 SPECIAL_CASES = ["no_process_noise", "no_observation", "precision_sum", "negative_decay", "mixed_zeros"]
 
 

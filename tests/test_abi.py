@@ -248,3 +248,42 @@ def test_size_overflow_is_rejected(lib):
                                  big, big, 1, 2, 16, 16 * P, 1 << 20, None) == 1
     assert lib.kla_layer_step(P, 2 * P, 3 * P, 4 * P, 0, 5 * P, 6 * P, 7 * P, 8 * P, 9 * P, None,
                               big, big, 2, 16, None) == 1
+
+
+def test_attention_and_lti_host_argument_errors(lib):
+    """The attention weights and the convolutional form reject bad arguments
+    on the host, before any CUDA call; empty problems are valid."""
+    P = 1 << 20  # fake pointers, never dereferenced
+    att = lib.kla_attention_weights
+    aargs = lambda **kw: [kw.get("a", P), kw.get("p", 2 * P), kw.get("dt", 0), kw.get("lam", 3 * P),
+                          kw.get("F", 8 * P), kw.get("B", 1), kw.get("T", 100), kw.get("H", 1), kw.get("N", 4),
+                          kw.get("t0", 0), kw.get("span", 100), kw.get("W", 16), None]
+    assert att(*aargs(W=0)) == 1
+    assert att(*aargs(W=65)) == 1                  # above KLA_ATTENTION_MAX_WINDOW
+    assert att(*aargs(t0=-1)) == 1
+    assert att(*aargs(t0=50, span=51)) == 1        # past the end of the sequence
+    assert att(*aargs(dt=4)) == 2
+    assert att(*aargs(lam=None)) == 1
+    assert att(*aargs(F=2 * P)) == 1               # F overlaps p
+    assert att(*aargs(span=0)) == 0                # empty
+    assert att(*aargs(B=0, a=None)) == 0
+    lti = lib.kla_scan_forward_lti
+    largs = lambda **kw: [kw.get("a", P), kw.get("phi", 2 * P), kw.get("b", 3 * P), kw.get("dt", 0),
+                          kw.get("lam0", 4 * P), kw.get("eta0", 5 * P), kw.get("lam", 6 * P),
+                          kw.get("eta", 7 * P), kw.get("mu", None), kw.get("var", None), kw.get("B", 1),
+                          kw.get("T", 4), kw.get("H", 1), kw.get("N", 4), kw.get("ws", 16 * P),
+                          kw.get("wsb", 1 << 20), None]
+    assert lti(*largs(B=-1)) == 1
+    assert lti(*largs(dt=2)) == 2
+    assert lti(*largs(a=None)) == 1
+    assert lti(*largs(eta=6 * P)) == 1             # eta_out overlaps lambda_out
+    assert lti(*largs(ws=2 * P)) == 1              # workspace overlaps phi
+    assert lti(*largs(ws=16 * P + 8)) == 6
+    assert lti(*largs(T=0)) == 0
+    out = ctypes.c_size_t(0)
+    assert lib.kla_scan_forward_lti_workspace_size(1, 65536, 32, 128, 0, ctypes.byref(out)) == 0
+    assert 0 < out.value < (1 << 20)               # run-boundary states only
+    assert lib.kla_scan_forward_lti_workspace_size(0, 1, 1, 1, 0, ctypes.byref(out)) == 0 and out.value == 0
+    k, n = ctypes.c_int(-1), ctypes.c_int(-1)
+    assert lib.kla_scan_forward_lti_plan(1, 65536, 1, 7, 0, P, P, ctypes.byref(k), ctypes.byref(n)) == 0
+    assert (k.value, n.value) == (1, 1)            # H*N = 7: one thread per channel
