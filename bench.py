@@ -313,14 +313,17 @@ def time_copy_bandwidth(device, steps: int = 20, nbytes: int = 4 << 30):
                    f"{steps} CUDA-event times"}
 
 
-def time_lti(kla, device, steps: int, warmup: int, peak: float):
+def time_lti(kla, device, steps: int, warmup: int, peak: float, tokens: int = 0):
     """The convolutional form (kla_scan_forward_lti) on the time-invariant
     workload, and the general scan on the same problem (a broadcast over
     time, p = 0) for comparison; each one's largest relative error of lambda
-    against the oracle's filter on 8 sampled whole channels."""
+    against the oracle's filter on 8 sampled whole channels.  ``tokens``
+    overrides T (smaller cases for profiler captures)."""
     import torch
     import oracle
     w = wl.LTI_WORKLOADS["lti"]
+    if tokens:
+        w = w.with_shape(T=tokens)
     x = wl.generate_lti(w)
     d = {k: torch.from_numpy(x[k]).to(device) for k in ("a", "phi", "b", "lam0", "eta0")}
     outs = [torch.empty((w.B, w.T, w.H, w.N), device=device) for _ in range(4)]
@@ -372,11 +375,14 @@ def time_lti(kla, device, steps: int, warmup: int, peak: float):
             "timing": "median of per-launch CUDA events (inputs of 2.1 GB, larger than L2)"}
 
 
-def time_attention(kla, device, steps: int, warmup: int, peak: float, W: int = 64):
+def time_attention(kla, device, steps: int, warmup: int, peak: float, W: int = 64, rows: int = 0):
     """kla_attention_weights over every window of W tokens of the LM-layer
-    workload (bf16 inputs), from the forward scan's lambda."""
+    workload (bf16 inputs), from the forward scan's lambda.  ``rows``
+    overrides B (smaller cases for profiler captures)."""
     import torch
     w = wl.WORKLOADS["lm_layer"]
+    if rows:
+        w = w.with_shape(B=rows)
     x = wl.generate(w)
     d = {k: torch.from_numpy(x[k]).to(device=device, dtype=torch.bfloat16) for k in wl.INPUT_NAMES}
     lam0 = torch.from_numpy(x["lam0"]).to(device)
@@ -760,9 +766,10 @@ def run_ours(args):
         del host_cfg
         if not args.no_forms:
             torch.cuda.empty_cache()
-            configs["lti"] = time_lti(kla, device, args.config_steps, args.warmup, peak)
+            configs["lti"] = time_lti(kla, device, args.config_steps, args.warmup, peak, tokens=args.tokens)
             torch.cuda.empty_cache()
-            configs["attention"] = time_attention(kla, device, args.config_steps, args.warmup, peak)
+            configs["attention"] = time_attention(kla, device, args.config_steps, args.warmup, peak,
+                                                  rows=args.attention_rows)
             torch.cuda.empty_cache()
             for name in ("lti", "attention"):
                 configs[name]["roofline"]["frac_of_same_run_copy"] = (configs[name]["gb_per_s"]
@@ -853,7 +860,10 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="long", choices=sorted(k for k, v in wl.WORKLOADS.items()
                                                                   if not v.decode))
     ap.add_argument("--tokens", type=int, default=0,
-                    help="override T (smaller cases for profiler captures; not a bench line)")
+                    help="override T of the headline and time-invariant workloads (smaller cases for "
+                         "profiler captures; not a bench line)")
+    ap.add_argument("--attention-rows", type=int, default=0,
+                    help="override B of the attention-weight leg (smaller cases for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--decode-replays", type=int, default=5)
     ap.add_argument("--ref-channels", type=int, default=256)

@@ -61,10 +61,17 @@ __device__ __forceinline__ Agg agg_identity() {
 // Rescale by 2^-e so that the largest Moebius entry lies in [1, 2).  A
 // multiplication by a power of two is exact, so the represented map -- and
 // every later rounding -- is unchanged: how often this runs does not change
-// any result bit (barring overflow).  The kernels run it every second token;
-// between two runs the largest entry grows at most by the square of the
-// largest row sum of M_t, so entries stay finite while
-// 1 + p phi + a^2 phi + p + a^2 < 2^63 per token.
+// any result bit (barring overflow).  The kernels run it every
+// KLA_RENORM_EVERY-th token (2 by default); between two runs the largest
+// entry grows at most by the largest row sum of M_t to that power, so
+// entries stay finite while 1 + p phi + a^2 phi + p + a^2 < 2^(126 /
+// KLA_RENORM_EVERY) per token (2^63 by default).
+#ifndef KLA_RENORM_EVERY
+#define KLA_RENORM_EVERY 2
+#endif
+constexpr int kRenormEvery = KLA_RENORM_EVERY;
+static_assert(kRenormEvery >= 1 && kRenormEvery <= 8, "renormalisation interval");
+__device__ __forceinline__ constexpr bool renorm_after(int t) { return (t + 1) % kRenormEvery == 0; }
 __device__ __forceinline__ void agg_renorm(Agg &g) {
     const float mx = fmaxf(fmaxf(fabsf(g.m11), fabsf(g.m12)), fmaxf(fabsf(g.m21), fabsf(g.m22)));
     int e = (__float_as_int(mx) >> 23) & 0xff;  // biased exponent of the max

@@ -78,6 +78,16 @@ struct StreamParams {
     int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
 };
 
+// What the producer tells the chunk warps about the chunk in a stage: its
+// work unit's tile coordinates and run bounds, computed once per unit, so
+// the chunk warps do no index division.
+struct StreamChunk {
+    int64_t tile;                  // bb * nct + ct
+    int chunk;                     // -1: no more work
+    int part, bb, ct;
+    int first, last;               // chunks of the run
+};
+
 template <typename Tin, int L, int W, int NS, int G>
 struct StreamTile {
     // Chunk j sits in stage j % NS and is handled by warp j % W.  With
@@ -94,8 +104,8 @@ struct StreamTile {
     static constexpr int OUTBUF_BYTES = 4 * OUTBOX_BYTES;           // four outputs
     static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][32] fp32
     static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][32] fp32
-    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: unit (int64), chunk (int64)
-    static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128); // full, empty, carry
+    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: StreamChunk
+    static constexpr int BAR_OFF = align_up(META_OFF + NS * (int)sizeof(StreamChunk), 128);  // full, empty, carry
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
 
@@ -116,8 +126,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     uint64_t *empty = full + NS;
     uint64_t *carry_bar = empty + NS;
     float *slots = reinterpret_cast<float *>(smem + Cfg::CARRY_OFF);
-    int64_t *meta_unit = reinterpret_cast<int64_t *>(smem + Cfg::META_OFF);  // -1: no more work
-    int64_t *meta_chunk = meta_unit + NS;
+    StreamChunk *meta = reinterpret_cast<StreamChunk *>(smem + Cfg::META_OFF);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -146,27 +155,30 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             }
             return s;
         };
-        auto load = [&](int64_t unit, int chunk, int bb, int ct) {
+        auto load = [&](const StreamChunk &m) {
             const int s = claim();
-            meta_unit[s] = unit;
-            meta_chunk[s] = chunk;
+            meta[s] = m;
             Tin *stage = reinterpret_cast<Tin *>(smem + s * Cfg::STAGE_BYTES);
             mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, chunk * L, bb, &full[s]);
+                tma_load_3d(stage + q * LC, &maps.in[q], m.ct * 32, m.chunk * L, m.bb, &full[s]);
         };
         // one unit: the tile's run u / ntiles, in time order (its tile
         // coordinates computed once per unit, not per chunk)
         auto unit_chunks = [&](int64_t u) {
-            const int64_t tile = u % prm.ntiles;
-            const int part = (int)(u / prm.ntiles);
-            const int bb = (int)(tile / prm.nct);
-            const int ct = (int)(tile - (int64_t)bb * prm.nct);
-            const int first = part * prm.chunks_per_part;
-            const int last = min(first + prm.chunks_per_part, prm.nchunks) - 1;
+            StreamChunk m;
+            m.tile = u % prm.ntiles;
+            m.part = (int)(u / prm.ntiles);
+            m.bb = (int)(m.tile / prm.nct);
+            m.ct = (int)(m.tile - (int64_t)m.bb * prm.nct);
+            m.first = m.part * prm.chunks_per_part;
+            m.last = min(m.first + prm.chunks_per_part, prm.nchunks) - 1;
 #pragma unroll 1
-            for (int c = first; c <= last; ++c) load(u, c, bb, ct);
+            for (int c = m.first; c <= m.last; ++c) {
+                m.chunk = c;
+                load(m);
+            }
         };
         if (prm.parts == 1) {
 #pragma unroll 1
@@ -183,7 +195,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 #pragma unroll 1
         for (int k = 0; k < W; ++k) {
             const int s = claim();
-            meta_unit[s] = -1;
+            meta[s].chunk = -1;
             mbar_arrive(&full[s]);
         }
         return;
@@ -197,21 +209,20 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     for (int64_t j = w;; j += W) {
         const int s = (int)(j % NS);
         mbar_wait_or_flag(&full[s], (unsigned)((j / NS) & 1), prm.wait_ns);
-        const int64_t unit = meta_unit[s];
-        if (unit < 0) break;
-        const int64_t chunk = meta_chunk[s];
-        const int64_t tile = unit % prm.ntiles;
-        const int64_t part = unit / prm.ntiles;
-        const int64_t bb = tile / prm.nct;
-        const int64_t ct = tile - bb * prm.nct;
+        const StreamChunk m = meta[s];
+        if (m.chunk < 0) break;
+        const int64_t chunk = m.chunk;
+        const int64_t tile = m.tile;
+        const int64_t part = m.part;
+        const int64_t bb = m.bb;
+        const int64_t ct = m.ct;
         const int64_t t0 = chunk * L;
         const int t_valid = (int)(prm.T - t0 < (int64_t)L ? prm.T - t0 : (int64_t)L);
         const int64_t ch = ct * 32 + lane;
         const bool cvalid = ch < prm.HN;
         const Tin *stage = reinterpret_cast<const Tin *>(smem + s * Cfg::STAGE_BYTES);
-        const int64_t first = part * prm.chunks_per_part;  // first chunk of this unit
-        const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
-                                                                         : (int64_t)prm.nchunks) - 1;
+        const int64_t first = m.first;  // chunks of this unit
+        const int64_t last = m.last;
 
         // State entering chunk j -- from the previous chunk's warp, from the
         // prior at a tile's first chunk, or from the previous run of the tile
@@ -312,7 +323,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 #pragma unroll
             for (int t = 0; t < L; ++t) {
                 agg_push_token(g, xa[t], xp[t], xf[t], xb[t]);
-                if (t & 1) agg_renorm(g);
+                if (renorm_after(t)) agg_renorm(g);
             }
             agg_renorm(g);
             // (2) carry
@@ -338,7 +349,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
                 const int i = t * 32 + lane;
                 agg_push_token(g, to_f32(stage[i]), to_f32(stage[LC + i]), to_f32(stage[2 * LC + i]),
                                to_f32(stage[3 * LC + i]));
-                if (t & 1) agg_renorm(g);
+                if (renorm_after(t)) agg_renorm(g);
             }
             agg_renorm(g);
             float lam, eta;

@@ -24,7 +24,8 @@
 // are below the TMA minimum), and writes only y and s.  The chunk warps form
 // the evidence in registers, run the chunk aggregate / carry / recursion of
 // the streaming kernel, and reduce the readout over the Ns lanes of a value
-// coordinate with warp shuffles.
+// coordinate through a per-warp transpose in shared memory (each lane then
+// sums whole rows for L / Ns tokens and stores their y and s).
 #pragma once
 
 #include "kla_forward_stream.cuh"
@@ -82,7 +83,13 @@ struct LayerTile {
     static constexpr int THREADS = 32 * (W + 1);
     static constexpr int CARRY_OFF = NS * STAGE_BYTES;                       // [W][2][32] fp32
     static constexpr int META_OFF = CARRY_OFF + W * 2 * 32 * 4;              // [NS] LayerChunk
-    static constexpr int BAR_OFF = align_up(META_OFF + NS * (int)sizeof(LayerChunk), 128);
+    // Readout transpose, per chunk warp: the q mu and q^2 var terms of a
+    // chunk, [2][L][TROW] fp32.  Rows are padded to 36 floats so that the
+    // 16-byte row reads of eight lanes (eight tokens) fall in distinct banks.
+    static constexpr int TROW = 36;
+    static constexpr int TBUF_BYTES = 2 * L * TROW * 4;
+    static constexpr int TBUF_OFF = align_up(META_OFF + NS * (int)sizeof(LayerChunk), 128);
+    static constexpr int BAR_OFF = align_up(TBUF_OFF + W * TBUF_BYTES, 128);
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
 
@@ -109,6 +116,24 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         :: "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)),
            "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Sum of M consecutive floats of shared memory (16-byte aligned), as a
+// pairwise tree of float4 reads.
+template <int M>
+__device__ __forceinline__ float row_sum(const float *src) {
+    static_assert(M % 4 == 0, "whole float4 reads");
+    float part[M / 4];
+#pragma unroll
+    for (int c = 0; c < M / 4; ++c) {
+        const float4 v = *reinterpret_cast<const float4 *>(src + 4 * c);
+        part[c] = (v.x + v.y) + (v.z + v.w);
+    }
+#pragma unroll
+    for (int step = 1; step < M / 4; step *= 2)
+#pragma unroll
+        for (int c = 0; c + step < M / 4; c += 2 * step) part[c] += part[c + step];
+    return part[0];
 }
 
 template <typename Tin, int NSX, int L, int W, int NS>
@@ -220,6 +245,8 @@ kla_layer_forward_kernel(const LayerParams prm, const __grid_constant__ LayerMap
     const int w = warp - 1;
     const int n = lane % NSX;          // state channel of the value coordinate
     const int dl = lane / NSX;         // value coordinate within the tile
+    float *ty = reinterpret_cast<float *>(smem + Cfg::TBUF_OFF + w * Cfg::TBUF_BYTES);  // [L][TROW]
+    float *ts = ty + L * Cfg::TROW;
     int s = w;
     unsigned par = 0;
     const int prev_w = w > 0 ? w - 1 : W - 1;
@@ -288,9 +315,8 @@ kla_layer_forward_kernel(const LayerParams prm, const __grid_constant__ LayerMap
                 if (lane == 0) st_release_gpu(prm.part_flags + slot, 1u);
             }
         };
-        // Readout of one token: sum over the Ns lanes of the value coordinate
-        // (two independent shuffle chains; folding both sums into one
-        // butterfly issued fewer instructions but measured 14% slower).
+        // Readout of one token of a ragged chunk: sum over the Ns lanes of the
+        // value coordinate with shuffles, stored by the coordinate's lane n = 0.
         auto readout = [&](int t, float q, const TokenOut &o) {
             float ym = q * o.mu;
             float sv2 = (q * q) * o.var;
@@ -330,13 +356,32 @@ kla_layer_forward_kernel(const LayerParams prm, const __grid_constant__ LayerMap
 #pragma unroll
             for (int t = 0; t < L; ++t) {
                 agg_push_token(g, a, p, xf[t], xb[t]);
-                if (t & 1) agg_renorm(g);
+                if (renorm_after(t)) agg_renorm(g);
             }
             agg_renorm(g);
             float lam = 0.f, eta = 0.f;
             chunk_carry(g, lam, eta);
+            // The readout of a full chunk, transposed: every lane writes its
+            // terms q mu and q^2 var of each token into the warp's buffer
+            // (one row per token), then lane (dl, n) sums row n + r Ns of its
+            // value coordinate dl for r = 0 .. L/Ns - 1 and stores y and s of
+            // those tokens -- L / Ns sums of Ns terms per lane instead of a
+            // shuffle butterfly per token.
 #pragma unroll
-            for (int t = 0; t < L; ++t) readout(t, xq[t], filter_token(lam, eta, a, p, xf[t], xb[t]));
+            for (int t = 0; t < L; ++t) {
+                const TokenOut o = filter_token(lam, eta, a, p, xf[t], xb[t]);
+                ty[t * Cfg::TROW + lane] = xq[t] * o.mu;
+                ts[t * Cfg::TROW + lane] = (xq[t] * xq[t]) * o.var;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < L / NSX; ++r) {
+                const int tok = r * NSX + n;
+                const float sy = row_sum<NSX>(ty + tok * Cfg::TROW + dl * NSX);
+                __stcs(yrow + tok * ystride, sy);
+                if (srow) __stcs(srow + tok * ystride, row_sum<NSX>(ts + tok * Cfg::TROW + dl * NSX));
+            }
+            __syncwarp();
             final_state(lam, eta);
         } else {
             // Ragged last chunk, straight from shared memory.
@@ -346,7 +391,7 @@ kla_layer_forward_kernel(const LayerParams prm, const __grid_constant__ LayerMap
                 const float kk = to_f32(sk[t * NSX + n]);
                 const float ww = to_f32(sw[t * DPW + dl]);
                 agg_push_token(g, a, p, (kk * kk) * ww, (kk * ww) * to_f32(sv[t * DPW + dl]));
-                if (t & 1) agg_renorm(g);
+                if (renorm_after(t)) agg_renorm(g);
             }
             agg_renorm(g);
             float lam = 0.f, eta = 0.f;

@@ -37,7 +37,8 @@
 // boxes stored with TMA.  Rows past T arrive as zeros (TMA fill) and are
 // clipped on store, so a ragged last chunk needs no separate path.  Tiles
 // that do not spread evenly over the SMs are cut into runs taken by ticket,
-// as in the general streaming scan; run boundaries hand on fp64 states.
+// as in the general streaming scan; run boundaries hand on fp64 states.  The
+// producer passes each chunk's tile coordinates in the stage's metadata.
 #pragma once
 
 #include "kla_forward_stream.cuh"
@@ -74,8 +75,8 @@ struct LtiTile {
     static constexpr int OUTBUF_BYTES = 4 * G * 32 * 4;               // four outputs, one group
     static constexpr int OUT_OFF = NS * STAGE_BYTES;                   // [W][2] output boxes
     static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES;   // [W][2][32] fp64
-    static constexpr int META_OFF = CARRY_OFF + W * 2 * 32 * 8;        // per stage: unit, chunk (int64)
-    static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128);
+    static constexpr int META_OFF = CARRY_OFF + W * 2 * 32 * 8;        // per stage: StreamChunk
+    static constexpr int BAR_OFF = align_up(META_OFF + NS * (int)sizeof(StreamChunk), 128);
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
 
@@ -122,8 +123,7 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
     uint64_t *empty = full + NS;
     uint64_t *carry_bar = empty + NS;
     double *slots = reinterpret_cast<double *>(smem + Cfg::CARRY_OFF);
-    int64_t *meta_unit = reinterpret_cast<int64_t *>(smem + Cfg::META_OFF);  // -1: no more work
-    int64_t *meta_chunk = meta_unit + NS;
+    StreamChunk *meta = reinterpret_cast<StreamChunk *>(smem + Cfg::META_OFF);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -153,21 +153,22 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
             return s;
         };
         auto unit_chunks = [&](int64_t u) {
-            const int64_t tile = u % prm.ntiles;
-            const int part = (int)(u / prm.ntiles);
-            const int bb = (int)(tile / prm.nct);
-            const int ct = (int)(tile - (int64_t)bb * prm.nct);
-            const int first = part * prm.chunks_per_part;
-            const int last = min(first + prm.chunks_per_part, prm.nchunks) - 1;
+            StreamChunk m;
+            m.tile = u % prm.ntiles;
+            m.part = (int)(u / prm.ntiles);
+            m.bb = (int)(m.tile / prm.nct);
+            m.ct = (int)(m.tile - (int64_t)m.bb * prm.nct);
+            m.first = m.part * prm.chunks_per_part;
+            m.last = min(m.first + prm.chunks_per_part, prm.nchunks) - 1;
 #pragma unroll 1
-            for (int c = first; c <= last; ++c) {
+            for (int c = m.first; c <= m.last; ++c) {
                 const int s = claim();
-                meta_unit[s] = u;
-                meta_chunk[s] = c;
+                m.chunk = c;
+                meta[s] = m;
                 Tin *stage = reinterpret_cast<Tin *>(smem + s * Cfg::STAGE_BYTES);
                 mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
-                tma_load_3d(stage, &maps.in[0], ct * 32, c * L, bb, &full[s]);
-                tma_load_3d(stage + LC, &maps.in[1], ct * 32, c * L, bb, &full[s]);
+                tma_load_3d(stage, &maps.in[0], m.ct * 32, c * L, m.bb, &full[s]);
+                tma_load_3d(stage + LC, &maps.in[1], m.ct * 32, c * L, m.bb, &full[s]);
             }
         };
         if (prm.parts == 1) {
@@ -184,7 +185,7 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
 #pragma unroll 1
         for (int k = 0; k < W; ++k) {
             const int s = claim();
-            meta_unit[s] = -1;
+            meta[s].chunk = -1;
             mbar_arrive(&full[s]);
         }
         return;
@@ -200,19 +201,18 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
     for (int64_t j = w;; j += W) {
         const int s = (int)(j % NS);
         mbar_wait_or_flag(&full[s], (unsigned)((j / NS) & 1), prm.wait_ns);
-        const int64_t unit = meta_unit[s];
-        if (unit < 0) break;
-        const int64_t chunk = meta_chunk[s];
-        const int64_t tile = unit % prm.ntiles;
-        const int64_t part = unit / prm.ntiles;
-        const int64_t bb = tile / prm.nct;
-        const int64_t ct = tile - bb * prm.nct;
+        const StreamChunk m = meta[s];
+        if (m.chunk < 0) break;
+        const int64_t chunk = m.chunk;
+        const int64_t tile = m.tile;
+        const int64_t part = m.part;
+        const int64_t bb = m.bb;
+        const int64_t ct = m.ct;
         const int64_t t0 = chunk * L;
         const int64_t ch = ct * 32 + lane;
         const bool cvalid = ch < prm.HN;
-        const int64_t first = part * prm.chunks_per_part;
-        const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
-                                                                         : (int64_t)prm.nchunks) - 1;
+        const int64_t first = m.first;
+        const int64_t last = m.last;
         if (tile != power_tile) {
             lti_powers<S, L>(cvalid ? (double)prm.a[bb * prm.HN + ch] : 1.0, kp);
             power_tile = tile;
