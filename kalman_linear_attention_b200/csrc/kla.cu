@@ -19,6 +19,7 @@
 #include "kla_backward.cuh"
 #include "kla_forward.cuh"
 #include "kla_forward_stream.cuh"
+#include "kla_forward_wide.cuh"
 #include "kla_attention.cuh"
 #include "kla_layer.cuh"
 #include "kla_lti.cuh"
@@ -108,8 +109,26 @@ constexpr int stream_stages() {
 }
 
 // 0: choose by shape; 1: the chunked kernel with cross-CTA carries; 2: the
-// channel-owning streaming kernel (test hook kla_debug_force_forward_kernel).
+// channel-owning streaming kernel; 3: the wide kernel, one warp per 32 x VEC
+// channels for the whole sequence (test hook kla_debug_force_forward_kernel).
 std::atomic<int> g_force_kernel{0};
+
+// Wide kernel: channels per lane, tokens of loads issued ahead of their
+// arithmetic, warps per CTA, and the fewest warps per SM (channel tiles of
+// 32 x VEC over the SM count) for which the shape picks it.
+#ifndef KLA_WIDE_VEC
+#define KLA_WIDE_VEC 4
+#endif
+#ifndef KLA_WIDE_D
+#define KLA_WIDE_D 4
+#endif
+#ifndef KLA_WIDE_WARPS
+#define KLA_WIDE_WARPS 4
+#endif
+#ifndef KLA_WIDE_MIN_WARPS_PER_SM
+#define KLA_WIDE_MIN_WARPS_PER_SM 6
+#endif
+constexpr int kWideVec = KLA_WIDE_VEC;
 
 constexpr size_t kHeaderBytes = 256;  // ticket counter + padding
 constexpr int kMaxGrid = 0x7fffffff;
@@ -336,6 +355,20 @@ int forward_kernel_choice(int64_t B, int64_t T, int64_t HN, size_t esz, const vo
                           const void *o3) {
     const int force = g_force_kernel.load();
     if (force == 1) return 1;
+    // 3: the wide kernel -- H*N a multiple of VEC, inputs aligned to VEC
+    // elements and outputs to VEC floats, and enough channel tiles to give
+    // every SM KLA_WIDE_MIN_WARPS_PER_SM warps (or the test hook forces it)
+    {
+        const auto al = [](const void *q, size_t bytes) {
+            return (reinterpret_cast<uintptr_t>(q) & (bytes - 1)) == 0;
+        };
+        const size_t ib = esz * kWideVec, ob = 4 * kWideVec;
+        const bool wide_geometry = HN % kWideVec == 0 && al(a, ib) && al(p, ib) && al(phi, ib) && al(b, ib) &&
+                                   al(o0, ob) && al(o1, ob) && al(o2, ob) && al(o3, ob);
+        const int64_t warps = B * ((HN + 32 * kWideVec - 1) / (32 * kWideVec));
+        if (wide_geometry && (force == 3 || (force == 0 && warps >= (int64_t)KLA_WIDE_MIN_WARPS_PER_SM * sm_count())))
+            return 3;
+    }
     const bool geometry = (HN * (int64_t)esz) % 16 == 0 && T >= kSL && HN >= 32 && aligned16(a) &&
                           aligned16(p) && aligned16(phi) && aligned16(b) && aligned16(o0) && aligned16(o1) &&
                           aligned16(o2) && aligned16(o3) && encode_fn() != nullptr;
@@ -448,9 +481,29 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
     const CUtensorMapDataType tdt =
         in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 
+    const int choice = forward_kernel_choice(B, T, HN, esz, a, p, phi, b, lambda_out, eta_out, mu_out, var_out);
+    if (choice == 3) {
+        kla::WideParams wp;
+        wp.in[0] = a; wp.in[1] = p; wp.in[2] = phi; wp.in[3] = b;
+        wp.lam0 = lambda0; wp.eta0 = eta0;
+        wp.out[0] = lambda_out; wp.out[1] = eta_out; wp.out[2] = mu_out; wp.out[3] = var_out;
+        wp.T = T; wp.HN = HN;
+        wp.nwt = (HN + 32 * kWideVec - 1) / (32 * kWideVec);
+        wp.nunits = B * wp.nwt;
+        const int64_t grid = (wp.nunits + KLA_WIDE_WARPS - 1) / KLA_WIDE_WARPS;
+        if (grid > kMaxGrid) return KLA_ERR_INVALID_ARG;
+        if (in_dtype == KLA_F32)
+            kla::kla_forward_wide_kernel<float, kWideVec, KLA_WIDE_D, KLA_WIDE_WARPS>
+                <<<(unsigned)grid, 32 * KLA_WIDE_WARPS, 0, st>>>(wp);
+        else
+            kla::kla_forward_wide_kernel<__nv_bfloat16, kWideVec, KLA_WIDE_D, KLA_WIDE_WARPS>
+                <<<(unsigned)grid, 32 * KLA_WIDE_WARPS, 0, st>>>(wp);
+        return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+    }
     // The channel-owning streaming kernel when forward_kernel_choice picks it
-    // (it needs no workspace); otherwise the chunked kernel below.
-    if (forward_kernel_choice(B, T, HN, esz, a, p, phi, b, lambda_out, eta_out, mu_out, var_out) == 2) {
+    // (it needs no workspace beyond its run splits); otherwise the chunked
+    // kernel below.
+    if (choice == 2) {
         FwdMaps smaps;
         std::memset(&smaps, 0, sizeof(smaps));
         const void *ins4[4] = {a, p, phi, b};
@@ -615,11 +668,12 @@ KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int6
     *launches = 2;  // chunked kernel: workspace clear + scan
     if (*kernel == 2)
         *launches = stream_parts(B * ((HN + 31) / 32), (T + kSL - 1) / kSL) > 1 ? 2 : 1;
+    if (*kernel == 3) *launches = 1;
     return KLA_OK;
 }
 
 KLA_API kla_status_t kla_debug_force_forward_kernel(int which) {
-    if (which < 0 || which > 2) return KLA_ERR_INVALID_ARG;
+    if (which < 0 || which > 3) return KLA_ERR_INVALID_ARG;
     g_force_kernel.store(which);
     return KLA_OK;
 }

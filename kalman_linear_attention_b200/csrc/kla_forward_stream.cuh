@@ -116,6 +116,10 @@ __device__ __forceinline__ void mbar_wait_or_flag(uint64_t *bar, unsigned parity
     }
 }
 
+#ifndef KLA_STREAM_SPLIT_AGG
+#define KLA_STREAM_SPLIT_AGG 0
+#endif
+
 template <typename Tin, int L, int W, int NS, int G>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
 kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMaps maps) {
@@ -318,13 +322,30 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
-            // (1) the chunk's aggregate (renormalised every second token)
+            // (1) the chunk's aggregate
+#if KLA_STREAM_SPLIT_AGG
+            // two independent chains, one per half chunk, then one product
+            Agg g0 = agg_identity(), g1 = agg_identity();
+#pragma unroll
+            for (int t = 0; t < L / 2; ++t) {
+                agg_push_token(g0, xa[t], xp[t], xf[t], xb[t]);
+                agg_push_token(g1, xa[L / 2 + t], xp[L / 2 + t], xf[L / 2 + t], xb[L / 2 + t]);
+                if (renorm_after(t)) {
+                    agg_renorm(g0);
+                    agg_renorm(g1);
+                }
+            }
+            agg_renorm(g0);
+            agg_renorm(g1);
+            Agg g = agg_compose(g1, g0);
+#else
             Agg g = agg_identity();
 #pragma unroll
             for (int t = 0; t < L; ++t) {
                 agg_push_token(g, xa[t], xp[t], xf[t], xb[t]);
                 if (renorm_after(t)) agg_renorm(g);
             }
+#endif
             agg_renorm(g);
             // (2) carry
             float lam, eta;

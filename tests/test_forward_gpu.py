@@ -17,10 +17,11 @@ def _kla():
     return kla
 
 
-@pytest.fixture(params=[1, 2], ids=["chunked", "stream"])
+@pytest.fixture(params=[1, 2, 3], ids=["chunked", "stream", "wide"])
 def kernel(request):
-    """Force one of the two forward kernels (1: chunks exchange carries through
-    the workspace; 2: channel-owning streaming kernel, where its geometry holds)."""
+    """Force one of the forward kernels (1: chunks exchange carries through
+    the workspace; 2: channel-owning streaming kernel; 3: one warp per 128
+    channels for the whole sequence -- 2 and 3 where their geometry holds)."""
     kla = _kla()
     kla.debug_force_forward_kernel(request.param)
     yield request.param
@@ -111,12 +112,14 @@ def test_kernels_agree_to_rounding():
     x = wl.generate(w)
     d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
     res = []
-    for which in (1, 2):
+    for which in (1, 2, 3):
         kla.debug_force_forward_kernel(which)
+        assert kla.forward_plan(d["a"], d["p"], d["phi"], d["b"])[0] == which
         o = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
         res.append({k: t.double().cpu().numpy() for k, t in zip(parity.OUTPUTS, o)})
     kla.debug_force_forward_kernel(0)
     parity.assert_parity(res[1], res[0], 2e-6, time_axis=1, what="stream vs chunked")
+    parity.assert_parity(res[2], res[0], 2e-6, time_axis=1, what="wide vs chunked")
 
 
 def test_workspace_contents_do_not_matter(kernel):
