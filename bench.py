@@ -482,12 +482,16 @@ def time_e2e(kla, w, host, steps: int):
     return dt, h2d, d2h
 
 
-def time_decode(kla, device, steps_tokens: int | None, replays: int):
-    """Decode workload: tokens replayed from a CUDA graph of kla_scan_step calls."""
+def time_decode(kla, device, steps_tokens: int | None, replays: int, batch: int | None = None):
+    """Decode workload: tokens replayed from a CUDA graph of kla_scan_step calls
+    (``batch`` overrides B: with a single sequence the time per token is the
+    fixed cost of one step, launch included)."""
     import torch
     w = wl.WORKLOADS["decode"]
     if steps_tokens is not None:
         w = w.with_shape(T=steps_tokens)
+    if batch is not None:
+        w = w.with_shape(B=batch)
     dev, _ = inputs_to_device(w, device, keep_host=False)
     steps = {k: dev.pop(k).transpose(0, 1).contiguous() for k in wl.INPUT_NAMES}  # [T, B, H, N]
     lam = dev["lam0"].clone()
@@ -725,6 +729,11 @@ def run_ours(args):
     decode = None
     if not args.no_decode:
         decode = time_decode(kla, device, None, args.decode_replays)
+        probe = time_decode(kla, device, None, args.decode_replays, batch=1)
+        decode["fixed_cost_probe"] = {
+            "us_per_token": probe["ms_per_token"] * 1e3, "channels": 32 * 128,
+            "note": "the same graph of 1024 kla_scan_step calls on one sequence (4096 channels, 16 KB of "
+                    "inputs per step): the fixed cost of a step, launch included"}
         decode["input_roofline"] = {
             "bound": "hbm", "achieved": decode["input_gb_per_s"], "peak": peak, "unit": "GB/s",
             "frac": decode["input_gb_per_s"] / peak,

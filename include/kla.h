@@ -44,7 +44,9 @@
  *   wait that ran out) are recorded on the device and reported by
  *   kla_get_error(); the affected outputs are NaN.
  * - Preconditions, not checked per element: p_t >= 0, phi_t >= 0,
- *   lambda_0 > 0, and a_t^2 + p_t lambda_{t-1} > 0 (e.g. a_t != 0 or p_t > 0).
+ *   lambda_0 > 0, and a_t^2 + p_t lambda_{t-1} > 0 (e.g. a_t != 0 or p_t > 0);
+ *   the row sums of M_t stay below 2^63 per token (1 + p phi + a^2 phi + p +
+ *   a^2; 2^31 for kla_layer_forward), which keeps the chunk aggregates finite.
  *   Any real a_t is allowed (only a_t^2 enters the precision; the sign of a_t
  *   enters the gate).  The state must stay within fp32 range: with p_t = 0
  *   and |a_t| < 1 the precision grows like a^(-2t) and overflows after about
@@ -368,6 +370,10 @@ kla_status_t kla_layer_forward_workspace_size(int64_t B, int64_t T, int64_t H, i
  *                 on with kla_scan_step), or both NULL
  *   workspace     at least kla_layer_forward_workspace_size(...) bytes,
  *                 256-byte aligned (NULL when that is 0)
+ *
+ * Precondition (besides the scan's): per token and state channel,
+ * 1 + p phi + a^2 phi + p + a^2 < 2^31 with phi = k^2 w (the kernel
+ * renormalises its chunk aggregates every fourth token).
  *
  * Supported shapes: Ns = 8 or 16 (the state expansions the review lists),
  * D a multiple of 32 / Ns; k, q, v, w 16-byte aligned.  Anything else returns

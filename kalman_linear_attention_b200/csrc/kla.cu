@@ -1215,8 +1215,11 @@ namespace {
 #ifndef KLA_LTI_S
 #define KLA_LTI_S 8
 #endif
+#ifndef KLA_LTI_G
+#define KLA_LTI_G 8
+#endif
 constexpr int kLtiL = 32;
-constexpr int kLtiG = 8;
+constexpr int kLtiG = KLA_LTI_G;
 
 template <typename Tin>
 constexpr int lti_stages() {

@@ -72,6 +72,10 @@ __device__ __forceinline__ Agg agg_identity() {
 constexpr int kRenormEvery = KLA_RENORM_EVERY;
 static_assert(kRenormEvery >= 1 && kRenormEvery <= 8, "renormalisation interval");
 __device__ __forceinline__ constexpr bool renorm_after(int t) { return (t + 1) % kRenormEvery == 0; }
+// The same with another interval E (E-th powers of the row sums must stay
+// below 2^126: row sums below 2^(126 / E) per token).
+template <int E>
+__device__ __forceinline__ constexpr bool renorm_after_every(int t) { return (t + 1) % E == 0; }
 __device__ __forceinline__ void agg_renorm(Agg &g) {
     const float mx = fmaxf(fmaxf(fabsf(g.m11), fabsf(g.m12)), fmaxf(fabsf(g.m21), fabsf(g.m22)));
     int e = (__float_as_int(mx) >> 23) & 0xff;  // biased exponent of the max

@@ -78,9 +78,9 @@ struct StreamParams {
     int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
 };
 
-// What the producer tells the chunk warps about the chunk in a stage: its
-// work unit's tile coordinates and run bounds, computed once per unit, so
-// the chunk warps do no index division.
+// What a producer tells its chunk warps about the chunk in a stage: the work
+// unit's tile coordinates and run bounds, computed once per unit (used by
+// the convolutional-form kernel).
 struct StreamChunk {
     int64_t tile;                  // bb * nct + ct
     int chunk;                     // -1: no more work
@@ -104,8 +104,8 @@ struct StreamTile {
     static constexpr int OUTBUF_BYTES = 4 * OUTBOX_BYTES;           // four outputs
     static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][32] fp32
     static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][32] fp32
-    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: StreamChunk
-    static constexpr int BAR_OFF = align_up(META_OFF + NS * (int)sizeof(StreamChunk), 128);  // full, empty, carry
+    static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: unit (int64), chunk (int64)
+    static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128); // full, empty, carry
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
 };
 
@@ -115,10 +115,6 @@ __device__ __forceinline__ void mbar_wait_or_flag(uint64_t *bar, unsigned parity
         (void)mbar_wait_bounded(bar, parity, limit_ns);
     }
 }
-
-#ifndef KLA_STREAM_SPLIT_AGG
-#define KLA_STREAM_SPLIT_AGG 0
-#endif
 
 template <typename Tin, int L, int W, int NS, int G>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
@@ -130,7 +126,8 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     uint64_t *empty = full + NS;
     uint64_t *carry_bar = empty + NS;
     float *slots = reinterpret_cast<float *>(smem + Cfg::CARRY_OFF);
-    StreamChunk *meta = reinterpret_cast<StreamChunk *>(smem + Cfg::META_OFF);
+    int64_t *meta_unit = reinterpret_cast<int64_t *>(smem + Cfg::META_OFF);  // -1: no more work
+    int64_t *meta_chunk = meta_unit + NS;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -159,30 +156,27 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             }
             return s;
         };
-        auto load = [&](const StreamChunk &m) {
+        auto load = [&](int64_t unit, int chunk, int bb, int ct) {
             const int s = claim();
-            meta[s] = m;
+            meta_unit[s] = unit;
+            meta_chunk[s] = chunk;
             Tin *stage = reinterpret_cast<Tin *>(smem + s * Cfg::STAGE_BYTES);
             mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                tma_load_3d(stage + q * LC, &maps.in[q], m.ct * 32, m.chunk * L, m.bb, &full[s]);
+                tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, chunk * L, bb, &full[s]);
         };
         // one unit: the tile's run u / ntiles, in time order (its tile
         // coordinates computed once per unit, not per chunk)
         auto unit_chunks = [&](int64_t u) {
-            StreamChunk m;
-            m.tile = u % prm.ntiles;
-            m.part = (int)(u / prm.ntiles);
-            m.bb = (int)(m.tile / prm.nct);
-            m.ct = (int)(m.tile - (int64_t)m.bb * prm.nct);
-            m.first = m.part * prm.chunks_per_part;
-            m.last = min(m.first + prm.chunks_per_part, prm.nchunks) - 1;
+            const int64_t tile = u % prm.ntiles;
+            const int part = (int)(u / prm.ntiles);
+            const int bb = (int)(tile / prm.nct);
+            const int ct = (int)(tile - (int64_t)bb * prm.nct);
+            const int first = part * prm.chunks_per_part;
+            const int last = min(first + prm.chunks_per_part, prm.nchunks) - 1;
 #pragma unroll 1
-            for (int c = m.first; c <= m.last; ++c) {
-                m.chunk = c;
-                load(m);
-            }
+            for (int c = first; c <= last; ++c) load(u, c, bb, ct);
         };
         if (prm.parts == 1) {
 #pragma unroll 1
@@ -199,7 +193,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 #pragma unroll 1
         for (int k = 0; k < W; ++k) {
             const int s = claim();
-            meta[s].chunk = -1;
+            meta_unit[s] = -1;
             mbar_arrive(&full[s]);
         }
         return;
@@ -213,20 +207,21 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     for (int64_t j = w;; j += W) {
         const int s = (int)(j % NS);
         mbar_wait_or_flag(&full[s], (unsigned)((j / NS) & 1), prm.wait_ns);
-        const StreamChunk m = meta[s];
-        if (m.chunk < 0) break;
-        const int64_t chunk = m.chunk;
-        const int64_t tile = m.tile;
-        const int64_t part = m.part;
-        const int64_t bb = m.bb;
-        const int64_t ct = m.ct;
+        const int64_t unit = meta_unit[s];
+        if (unit < 0) break;
+        const int64_t chunk = meta_chunk[s];
+        const int64_t tile = unit % prm.ntiles;
+        const int64_t part = unit / prm.ntiles;
+        const int64_t bb = tile / prm.nct;
+        const int64_t ct = tile - bb * prm.nct;
         const int64_t t0 = chunk * L;
         const int t_valid = (int)(prm.T - t0 < (int64_t)L ? prm.T - t0 : (int64_t)L);
         const int64_t ch = ct * 32 + lane;
         const bool cvalid = ch < prm.HN;
         const Tin *stage = reinterpret_cast<const Tin *>(smem + s * Cfg::STAGE_BYTES);
-        const int64_t first = m.first;  // chunks of this unit
-        const int64_t last = m.last;
+        const int64_t first = part * prm.chunks_per_part;  // first chunk of this unit
+        const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
+                                                                         : (int64_t)prm.nchunks) - 1;
 
         // State entering chunk j -- from the previous chunk's warp, from the
         // prior at a tile's first chunk, or from the previous run of the tile
@@ -322,30 +317,13 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
-            // (1) the chunk's aggregate
-#if KLA_STREAM_SPLIT_AGG
-            // two independent chains, one per half chunk, then one product
-            Agg g0 = agg_identity(), g1 = agg_identity();
-#pragma unroll
-            for (int t = 0; t < L / 2; ++t) {
-                agg_push_token(g0, xa[t], xp[t], xf[t], xb[t]);
-                agg_push_token(g1, xa[L / 2 + t], xp[L / 2 + t], xf[L / 2 + t], xb[L / 2 + t]);
-                if (renorm_after(t)) {
-                    agg_renorm(g0);
-                    agg_renorm(g1);
-                }
-            }
-            agg_renorm(g0);
-            agg_renorm(g1);
-            Agg g = agg_compose(g1, g0);
-#else
+            // (1) the chunk's aggregate (renormalised every second token)
             Agg g = agg_identity();
 #pragma unroll
             for (int t = 0; t < L; ++t) {
                 agg_push_token(g, xa[t], xp[t], xf[t], xb[t]);
                 if (renorm_after(t)) agg_renorm(g);
             }
-#endif
             agg_renorm(g);
             // (2) carry
             float lam, eta;
