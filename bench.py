@@ -260,7 +260,8 @@ def time_launches(fn, steps: int, warmup: int, flush=None):
 
 
 FORWARD_KERNELS = {1: "kla_forward_kernel (chunked, cross-CTA carries; + its workspace clear kernel)",
-                   2: "kla_forward_stream_kernel (channel-owning streaming)"}
+                   2: "kla_forward_stream_kernel (channel-owning streaming)",
+                   3: "kla_forward_wide_kernel (one warp per channel tile, per-warp TMA ring)"}
 
 
 def time_config(kla, w: wl.Workload, device, steps: int, warmup: int, peak: float, flush):
@@ -690,8 +691,7 @@ def run_ours(args):
     sampler.start()
     total_ms, per_launch, plan, fwd_outs = time_forward(kla, w, dev, args.steps, args.warmup,
                                                         dist if world > 1 else None)
-    kernel_name = {1: "kla_forward_kernel (chunked; + its workspace clear kernel, timed together)",
-                   2: "kla_forward_stream_kernel (channel-owning streaming)"}[plan[0]]
+    kernel_name = FORWARD_KERNELS[plan[0]]
     clocks = sampler.stop()
 
     max_ms = max_over_ranks(total_ms, dist if world > 1 else None)

@@ -2,123 +2,130 @@
 // (sm_100a).
 //
 // When the channels alone give every SM several warps of work, the scan
-// needs no token-parallel machinery at all: one warp walks VEC x 32
-// consecutive channels of one batch row through the whole sequence, lane =
-// VEC channels, applying the plain per-token recursion of kla_device.cuh
-// (filter_token) token after token.  Each lane thus runs VEC independent
-// recursion chains side by side, its loads of a, p, phi, b and its streaming
-// stores of lambda, eta, mu, var are 4 x VEC bytes wide (fully used 128-byte
-// lines across the warp), and the loads of D tokens are issued before their
-// arithmetic so that D x 4 x 32 x VEC x elem bytes per warp are in flight.
-// There is no chunk aggregate, no carry, no shared memory and no wait: per
-// token-channel it issues roughly a quarter of the instructions of the
-// chunked kernels, and every byte crosses HBM once.  The results are the
-// per-token recursion from the prior, exactly as the other kernels' second
-// pass computes it.
+// needs no token-parallel machinery: one warp walks a tile of CW channels of
+// one batch row through the whole sequence with the plain per-token
+// recursion of kla_device.cuh (filter_token), lane = channel.  Without chunk
+// aggregates or carries, a token costs one pass instead of the chunked
+// kernels' two.
+//
+// What such a kernel needs is bytes in flight: a warp streams its tile
+// through its own ring of NSTG shared-memory stages of L tokens, each filled
+// by TMA bulk-tensor loads (box {CW, L, 1} of a, p, phi, b) that lane 0
+// issues NSTG chunks ahead and that complete on the stage's mbarrier.  After
+// a chunk's L tokens the warp refills the stage with the chunk NSTG ahead of
+// it in its own sequence of (unit, chunk) items.  Outputs leave as direct
+// coalesced stores from registers (CW x 4 bytes per output and token).
+//
+// CW is 32 (fp32 inputs: a 128-byte row per input and token) or 16 (bf16
+// inputs: 32 bytes, one sector, so that a batch of B x H*N / 16 tiles still
+// gives every SM its warps); with CW = 16 the upper half-warp idles, which
+// costs issue slots the kernel has to spare.  Units (batch row, channel
+// tile) are dealt to the grid's CTAs round-robin and, inside a CTA, to its
+// warps; rows past T arrive as zeros from TMA and are not stored; lanes past
+// H*N load zeros and store nothing.  Every wait is bounded.
 #pragma once
 
-#include "kla_device.cuh"
+#include "kla_forward_stream.cuh"
 
 namespace kla {
 
 struct WideParams {
-    const void *in[4];             // a, p, phi, b [B, T, H, N]
     const float *lam0, *eta0;      // [B, H, N]
     float *out[4];                 // lambda, eta, mu, var; mu / var may be null
     int64_t T, HN;
-    int64_t nwt;                   // warp tiles (of 32 x VEC channels) per batch row
-    int64_t nunits;                // B * nwt
+    int64_t ntile;                 // channel tiles per batch row: ceil(HN / CW)
+    int64_t nunits;                // B * ntile
+    int nchunks;                   // ceil(T / L)
+    uint64_t wait_ns;
 };
 
-// VEC consecutive values of an input at element index i (i a multiple of
-// VEC), widened to fp32; streaming (evict-first) loads.
-template <typename Tin, int VEC> struct WideLd;
-template <> struct WideLd<float, 4> {
-    static __device__ __forceinline__ void load(const void *p, int64_t i, float (&v)[4]) {
-        const float4 x = __ldcs(reinterpret_cast<const float4 *>(static_cast<const float *>(p) + i));
-        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-    }
-};
-template <> struct WideLd<float, 2> {
-    static __device__ __forceinline__ void load(const void *p, int64_t i, float (&v)[2]) {
-        const float2 x = __ldcs(reinterpret_cast<const float2 *>(static_cast<const float *>(p) + i));
-        v[0] = x.x; v[1] = x.y;
-    }
-};
-template <> struct WideLd<__nv_bfloat16, 4> {
-    static __device__ __forceinline__ void load(const void *p, int64_t i, float (&v)[4]) {
-        const uint2 u = __ldcs(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p) + i));
-        v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
-        v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
-    }
-};
-template <> struct WideLd<__nv_bfloat16, 2> {
-    static __device__ __forceinline__ void load(const void *p, int64_t i, float (&v)[2]) {
-        const unsigned u = __ldcs(reinterpret_cast<const unsigned *>(static_cast<const __nv_bfloat16 *>(p) + i));
-        v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xffff0000u);
-    }
+template <typename Tin, int CW, int L, int NSTG, int NWARP>
+struct WideTile {
+    static constexpr int STAGE_BYTES = 4 * L * CW * (int)sizeof(Tin);  // [4][L][CW]
+    static_assert(STAGE_BYTES % 128 == 0, "stages stay 128-byte aligned");
+    static constexpr int WARP_BYTES = NSTG * STAGE_BYTES;
+    static constexpr int BAR_OFF = NWARP * WARP_BYTES;                // [NWARP][NSTG] mbarriers
+    static constexpr int SMEM = align_up(BAR_OFF + NWARP * NSTG * 8, 128);
 };
 
-template <int VEC> struct WideSt;
-template <> struct WideSt<4> {
-    static __device__ __forceinline__ void store(float *p, int64_t i, const float (&v)[4]) {
-        __stcs(reinterpret_cast<float4 *>(p + i), make_float4(v[0], v[1], v[2], v[3]));
-    }
-};
-template <> struct WideSt<2> {
-    static __device__ __forceinline__ void store(float *p, int64_t i, const float (&v)[2]) {
-        __stcs(reinterpret_cast<float2 *>(p + i), make_float2(v[0], v[1]));
-    }
-};
-
-// One warp per (batch row, tile of 32 x VEC channels); WARPS warps per CTA.
-// Needs H*N % VEC == 0 and every array aligned to 4 x VEC bytes (2 x VEC for
-// bf16 inputs).
-template <typename Tin, int VEC, int D, int WARPS>
-__global__ void __launch_bounds__(32 * WARPS) kla_forward_wide_kernel(const WideParams prm) {
-    const int64_t unit = (int64_t)blockIdx.x * WARPS + (threadIdx.x >> 5);
-    if (unit >= prm.nunits) return;
+template <typename Tin, int CW, int L, int NSTG, int NWARP>
+__global__ void __launch_bounds__(32 * NWARP, 1)
+kla_forward_wide_kernel(const WideParams prm, const __grid_constant__ FwdMaps maps) {
+    using Cfg = WideTile<Tin, CW, L, NSTG, NWARP>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t bb = unit / prm.nwt;
-    const int64_t c = (unit - bb * prm.nwt) * (32 * VEC) + lane * VEC;
-    if (c >= prm.HN) return;  // whole vectors: H*N is a multiple of VEC
-    float lam[VEC], eta[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) {  // the prior: scalar loads (its alignment is not checked)
-        lam[v] = prm.lam0[bb * prm.HN + c + v];
-        eta[v] = prm.eta0[bb * prm.HN + c + v];
+    unsigned char *ring = smem + w * Cfg::WARP_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::BAR_OFF) + w * NSTG;
+    if (lane == 0) {
+        for (int s = 0; s < NSTG; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
     }
-    const int64_t base = bb * prm.T * prm.HN + c;
-    float *const lo = prm.out[0], *const eo = prm.out[1], *const mo = prm.out[2], *const vo = prm.out[3];
-#pragma unroll 1
-    for (int64_t t0 = 0; t0 < prm.T; t0 += D) {
-        const int n = (int)(prm.T - t0 < D ? prm.T - t0 : D);
-        float xa[D][VEC], xp[D][VEC], xf[D][VEC], xb[D][VEC];
+    __syncwarp();
+
+    // This warp's units: u = blockIdx.x + gridDim.x * (w + NWARP * k), k = 0, 1, ...
+    const int64_t ustep = (int64_t)gridDim.x * NWARP;
+    const int64_t ufirst = blockIdx.x + (int64_t)gridDim.x * w;
+    // item i of the warp = chunk (i % nchunks) of its (i / nchunks)-th unit
+    const int64_t nitems = ufirst < prm.nunits ? ((prm.nunits - 1 - ufirst) / ustep + 1) * prm.nchunks : 0;
+    auto issue = [&](int64_t item) {  // lane 0: the TMA loads of one item into its stage
+        const int64_t u = ufirst + (item / prm.nchunks) * ustep;
+        const int chunk = (int)(item % prm.nchunks);
+        const int bb = (int)(u / prm.ntile);
+        const int ct = (int)(u - (int64_t)bb * prm.ntile);
+        const int s = (int)(item % NSTG);
+        Tin *stage = reinterpret_cast<Tin *>(ring + s * Cfg::STAGE_BYTES);
+        mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
 #pragma unroll
-        for (int u = 0; u < D; ++u) {
-            if (u < n) {
-                const int64_t i = base + (t0 + u) * prm.HN;
-                WideLd<Tin, VEC>::load(prm.in[0], i, xa[u]);
-                WideLd<Tin, VEC>::load(prm.in[1], i, xp[u]);
-                WideLd<Tin, VEC>::load(prm.in[2], i, xf[u]);
-                WideLd<Tin, VEC>::load(prm.in[3], i, xb[u]);
+        for (int q = 0; q < 4; ++q)
+            tma_load_3d(stage + q * L * CW, &maps.in[q], ct * CW, chunk * L, bb, &full[s]);
+    };
+    if (lane == 0)
+        for (int64_t i = 0; i < NSTG && i < nitems; ++i) issue(i);
+
+    float lam = 0.f, eta = 0.f;
+    int64_t chan = 0, row0 = 0;  // this lane's channel and the element index of token 0 of its unit
+    bool active = false;
+#pragma unroll 1
+    for (int64_t item = 0; item < nitems; ++item) {
+        const int chunk = (int)(item % prm.nchunks);
+        if (chunk == 0) {  // a new unit: its prior
+            const int64_t u = ufirst + (item / prm.nchunks) * ustep;
+            const int64_t bb = u / prm.ntile;
+            const int64_t ct = u - bb * prm.ntile;
+            chan = ct * CW + lane;
+            active = lane < CW && chan < prm.HN;
+            row0 = bb * prm.T * prm.HN + chan;
+            lam = active ? prm.lam0[bb * prm.HN + chan] : 1.f;
+            eta = active ? prm.eta0[bb * prm.HN + chan] : 0.f;
+        }
+        const int s = (int)(item % NSTG);
+        mbar_wait_or_flag(&full[s], (unsigned)((item / NSTG) & 1), prm.wait_ns);
+        const Tin *stage = reinterpret_cast<const Tin *>(ring + s * Cfg::STAGE_BYTES);
+        const int64_t t0 = (int64_t)chunk * L;
+        const int nv = (int)(prm.T - t0 < L ? prm.T - t0 : L);
+        const int c = lane < CW ? lane : 0;  // idle lanes of a half warp read lane 0's column
+        float *o0 = prm.out[0] + row0 + t0 * prm.HN;
+        float *o1 = prm.out[1] + row0 + t0 * prm.HN;
+        float *o2 = prm.out[2] ? prm.out[2] + row0 + t0 * prm.HN : nullptr;
+        float *o3 = prm.out[3] ? prm.out[3] + row0 + t0 * prm.HN : nullptr;
+#pragma unroll 4
+        for (int t = 0; t < nv; ++t) {
+            const int i = t * CW + c;
+            const TokenOut o = filter_token(lam, eta, to_f32(stage[i]), to_f32(stage[L * CW + i]),
+                                            to_f32(stage[2 * L * CW + i]), to_f32(stage[3 * L * CW + i]));
+            if (active) {
+                const int64_t off = (int64_t)t * prm.HN;
+                __stcs(o0 + off, o.lam);
+                __stcs(o1 + off, o.eta);
+                if (o2) __stcs(o2 + off, o.mu);
+                if (o3) __stcs(o3 + off, o.var);
             }
         }
-#pragma unroll
-        for (int u = 0; u < D; ++u) {
-            if (u < n) {
-                float ol[VEC], oe[VEC], om[VEC], ov[VEC];
-#pragma unroll
-                for (int v = 0; v < VEC; ++v) {
-                    const TokenOut o = filter_token(lam[v], eta[v], xa[u][v], xp[u][v], xf[u][v], xb[u][v]);
-                    ol[v] = o.lam; oe[v] = o.eta; om[v] = o.mu; ov[v] = o.var;
-                }
-                const int64_t i = base + (t0 + u) * prm.HN;
-                WideSt<VEC>::store(lo, i, ol);
-                WideSt<VEC>::store(eo, i, oe);
-                if (mo != nullptr) WideSt<VEC>::store(mo, i, om);
-                if (vo != nullptr) WideSt<VEC>::store(vo, i, ov);
-            }
+        __syncwarp();  // every lane has read the stage
+        if (lane == 0 && item + NSTG < nitems) {
+            fence_proxy_async_smem();  // the warp's reads of the stage before the copy that refills it
+            issue(item + NSTG);
         }
     }
 }

@@ -226,10 +226,12 @@ def test_bitwise_reproducible(kernel):
 
 
 def test_plan_matches_workloads():
-    """On a B200 the standard workloads take the streaming kernel except the
-    tiny one (2 tiles of 32 channels cannot occupy the GPU)."""
+    """On a B200: the tiny workload (2 tiles of 32 channels cannot occupy the
+    GPU) takes the chunked kernel, the long one (4096 channels) the streaming
+    kernel, and the LM-layer and stiff ones (1024 and 4096 channel tiles:
+    several warps per SM) the wide kernel."""
     kla = _kla()
-    for name, expect in (("tiny", 1), ("lm_layer", 2), ("long", 2), ("stiff", 2)):
+    for name, expect in (("tiny", 1), ("lm_layer", 3), ("long", 2), ("stiff", 3)):
         w = wl.WORKLOADS[name]
         dt = parity.torch_dtype(w)
         z = torch.empty((w.B, w.T, w.H, w.N), dtype=dt, device=DEV)
