@@ -260,8 +260,7 @@ def time_launches(fn, steps: int, warmup: int, flush=None):
 
 
 FORWARD_KERNELS = {1: "kla_forward_kernel (chunked, cross-CTA carries; + its workspace clear kernel)",
-                   2: "kla_forward_stream_kernel (channel-owning streaming)",
-                   3: "kla_forward_wide_kernel (one warp per channel tile, per-warp TMA ring)"}
+                   2: "kla_forward_stream_kernel (channel-owning streaming)"}
 
 
 def time_config(kla, w: wl.Workload, device, steps: int, warmup: int, peak: float, flush):
@@ -309,9 +308,14 @@ def time_copy_bandwidth(device, steps: int = 20, nbytes: int = 4 << 30):
     per = time_launches(lambda: dst.copy_(src), steps, 3)
     ms = statistics.median(per)
     del src, dst
+    dst2 = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+    per_w = time_launches(lambda: dst2.fill_(0.5), steps, 3)
+    ms_w = statistics.median(per_w)
+    del dst2
     return {"gb_per_s": 2 * nbytes / (ms * 1e-3) / 1e9, "ms": ms,
+            "write_only_gb_per_s": nbytes / (ms_w * 1e-3) / 1e9,
             "how": "torch copy_ of a 4 GiB fp32 buffer on the device, (read + write bytes) / median of "
-                   f"{steps} CUDA-event times"}
+                   f"{steps} CUDA-event times; write_only: torch fill_ of 4 GiB, bytes / median time"}
 
 
 def time_lti(kla, device, steps: int, warmup: int, peak: float, tokens: int = 0):

@@ -133,12 +133,10 @@ kla_status_t kla_scan_forward(const void *a, const void *p, const void *phi, con
  * shape and dtype with these input pointers (only their alignment matters;
  * they are not dereferenced), written to *kernel: 1 = the chunked kernel whose
  * chunks exchange carries through the workspace, 2 = the channel-owning
- * streaming kernel, 3 = the wide kernel (one warp walks 128 channels through
- * the whole sequence; chosen when B*H*N gives every SM several such warps);
- * *launches = the kernel launches one call enqueues (2 for the chunked
- * kernel, preceded by a workspace clear; 1 or 2 for the streaming kernel,
- * 2 when it splits tiles into runs; 1 for the wide kernel).  0 and 0 for an
- * empty problem.  Honours kla_debug_force_forward_kernel.
+ * streaming kernel; *launches = the kernel launches one call enqueues (2 for
+ * the chunked kernel, preceded by a workspace clear; 1 or 2 for the
+ * streaming kernel, 2 when it splits tiles into runs).  0 and 0 for an empty
+ * problem.  Honours kla_debug_force_forward_kernel.
  */
 kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
                                    const void *a, const void *p, const void *phi, const void *b,
@@ -150,11 +148,9 @@ kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int64_t N, k
  * exchange carries through the workspace (any shape); 2: the channel-owning
  * streaming kernel (used only when its geometry holds: 16-byte aligned
  * inputs, H*N*elem a multiple of 16 bytes, H*N >= 32, T >= 32; otherwise the
- * chunked kernel runs); 3: the wide kernel (used only when H*N is a multiple
- * of 4 and the arrays are aligned to 4 elements; otherwise the chunked
- * kernel runs).  All compute the same filter; their chunkings differ, so
- * results agree to rounding, not bit for bit.  KLA_ERR_INVALID_ARG for other
- * values.
+ * chunked kernel runs).  Both compute the same filter; their chunkings
+ * differ, so results agree to rounding, not bit for bit.  KLA_ERR_INVALID_ARG
+ * for other values.
  */
 kla_status_t kla_debug_force_forward_kernel(int which);
 

@@ -19,7 +19,6 @@
 #include "kla_backward.cuh"
 #include "kla_forward.cuh"
 #include "kla_forward_stream.cuh"
-#include "kla_forward_wide.cuh"
 #include "kla_attention.cuh"
 #include "kla_layer.cuh"
 #include "kla_lti.cuh"
@@ -109,31 +108,9 @@ constexpr int stream_stages() {
 }
 
 // 0: choose by shape; 1: the chunked kernel with cross-CTA carries; 2: the
-// channel-owning streaming kernel; 3: the wide kernel, one warp per channel
-// tile for the whole sequence (test hook kla_debug_force_forward_kernel).
+// channel-owning streaming kernel (test hook kla_debug_force_forward_kernel).
 std::atomic<int> g_force_kernel{0};
 
-// Wide kernel: channels per warp (32 for fp32 inputs, 16 for bf16), ring
-// stages per warp and warps per CTA (192 KB of stages per CTA either way),
-// and the fewest units (batch row x channel tile) per SM for which the shape
-// picks it.
-#ifndef KLA_WIDE_STAGES_F32
-#define KLA_WIDE_STAGES_F32 2
-#endif
-#ifndef KLA_WIDE_WARPS_F32
-#define KLA_WIDE_WARPS_F32 6
-#endif
-#ifndef KLA_WIDE_STAGES_BF16
-#define KLA_WIDE_STAGES_BF16 6
-#endif
-#ifndef KLA_WIDE_WARPS_BF16
-#define KLA_WIDE_WARPS_BF16 8
-#endif
-#ifndef KLA_WIDE_MIN_UNITS_PER_SM
-#define KLA_WIDE_MIN_UNITS_PER_SM 6
-#endif
-constexpr int kWideL = 32;
-int wide_cw(size_t esz) { return esz == 4 ? 32 : 16; }
 
 constexpr size_t kHeaderBytes = 256;  // ticket counter + padding
 constexpr int kMaxGrid = 0x7fffffff;
@@ -308,36 +285,6 @@ bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [B, T, HN] tensor viewed as dims {HN, T, B}, box {box_x, rows, 1}.
-bool encode_box_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz, int64_t B, int64_t T,
-                    int64_t HN, int box_x, int rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)HN, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[2] = {(cuuint64_t)(HN * esz), (cuuint64_t)(T * HN * esz)};
-    const cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)rows, 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <typename Tin>
-cudaError_t launch_wide(const kla::WideParams &prm, const FwdMaps &maps, cudaStream_t stream) {
-    constexpr bool f32 = sizeof(Tin) == 4;
-    constexpr int CW = f32 ? 32 : 16;
-    constexpr int NSTG = f32 ? KLA_WIDE_STAGES_F32 : KLA_WIDE_STAGES_BF16;
-    constexpr int NWARP = f32 ? KLA_WIDE_WARPS_F32 : KLA_WIDE_WARPS_BF16;
-    using Cfg = kla::WideTile<Tin, CW, kWideL, NSTG, NWARP>;
-    static_assert(Cfg::SMEM <= 227 * 1024, "wide kernel shared memory");
-    auto kernel = kla::kla_forward_wide_kernel<Tin, CW, kWideL, NSTG, NWARP>;
-    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = std::min<int64_t>((prm.nunits + NWARP - 1) / NWARP, sm_count());
-    kernel<<<(unsigned)grid, 32 * NWARP, Cfg::SMEM, stream>>>(prm, maps);
-    return cudaGetLastError();
-}
-
 // Runs per tile for the streaming kernel: the number P <= KLA_STREAM_MAX_PARTS
 // of runs per tile whose units (tiles x P) fill the SMs' rounds best, among
 // those that keep at least 8 chunks per run; 1 when there are fewer than two
@@ -390,19 +337,6 @@ int forward_kernel_choice(int64_t B, int64_t T, int64_t HN, size_t esz, const vo
                           const void *o3) {
     const int force = g_force_kernel.load();
     if (force == 1) return 1;
-    // 3: the wide kernel -- its TMA geometry holds (16-byte aligned inputs,
-    // H*N*elem a multiple of 16 bytes, H*N >= 16) and the channel tiles give
-    // every SM KLA_WIDE_MIN_UNITS_PER_SM warps of work (or the test hook
-    // forces it); it stores outputs with plain loads, any alignment
-    {
-        const bool wide_geometry = (HN * (int64_t)esz) % 16 == 0 && HN >= 16 && aligned16(a) && aligned16(p) &&
-                                   aligned16(phi) && aligned16(b) && encode_fn() != nullptr;
-        const int cw = wide_cw(esz);
-        const int64_t units = B * ((HN + cw - 1) / cw);
-        if (wide_geometry &&
-            (force == 3 || (force == 0 && units >= (int64_t)KLA_WIDE_MIN_UNITS_PER_SM * sm_count())))
-            return 3;
-    }
     const bool geometry = (HN * (int64_t)esz) % 16 == 0 && T >= kSL && HN >= 32 && aligned16(a) &&
                           aligned16(p) && aligned16(phi) && aligned16(b) && aligned16(o0) && aligned16(o1) &&
                           aligned16(o2) && aligned16(o3) && encode_fn() != nullptr;
@@ -516,27 +450,6 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
         in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 
     const int choice = forward_kernel_choice(B, T, HN, esz, a, p, phi, b, lambda_out, eta_out, mu_out, var_out);
-    if (choice == 3) {
-        const int cw = wide_cw(esz);
-        FwdMaps wmaps;
-        std::memset(&wmaps, 0, sizeof(wmaps));
-        const void *ins4[4] = {a, p, phi, b};
-        bool ok = true;
-        for (int k = 0; k < 4 && ok; ++k) ok = encode_box_map(&wmaps.in[k], ins4[k], tdt, esz, B, T, HN, cw, kWideL);
-        if (ok) {
-            kla::WideParams wp;
-            wp.lam0 = lambda0; wp.eta0 = eta0;
-            wp.out[0] = lambda_out; wp.out[1] = eta_out; wp.out[2] = mu_out; wp.out[3] = var_out;
-            wp.T = T; wp.HN = HN;
-            wp.ntile = (HN + cw - 1) / cw;
-            wp.nunits = B * wp.ntile;
-            wp.nchunks = (int)((T + kWideL - 1) / kWideL);
-            wp.wait_ns = g_wait_ns.load();
-            const cudaError_t e = in_dtype == KLA_F32 ? launch_wide<float>(wp, wmaps, st)
-                                                      : launch_wide<__nv_bfloat16>(wp, wmaps, st);
-            return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
-        }
-    }
     // The channel-owning streaming kernel when forward_kernel_choice picks it
     // (it needs no workspace beyond its run splits); otherwise the chunked
     // kernel below.
@@ -554,6 +467,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
         if (ok) {
             kla::StreamParams sp;
             sp.lam0 = lambda0; sp.eta0 = eta0;
+            sp.out[0] = lambda_out; sp.out[1] = eta_out; sp.out[2] = mu_out; sp.out[3] = var_out;
             sp.write_mu = mu_out != nullptr; sp.write_var = var_out != nullptr;
             sp.T = T; sp.HN = HN; sp.ntiles = B * ((HN + 31) / 32);
             sp.nct = (int)((HN + 31) / 32);
@@ -705,12 +619,11 @@ KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int6
     *launches = 2;  // chunked kernel: workspace clear + scan
     if (*kernel == 2)
         *launches = stream_parts(B * ((HN + 31) / 32), (T + kSL - 1) / kSL) > 1 ? 2 : 1;
-    if (*kernel == 3) *launches = 1;
     return KLA_OK;
 }
 
 KLA_API kla_status_t kla_debug_force_forward_kernel(int which) {
-    if (which < 0 || which > 3) return KLA_ERR_INVALID_ARG;
+    if (which < 0 || which > 2) return KLA_ERR_INVALID_ARG;
     g_force_kernel.store(which);
     return KLA_OK;
 }
@@ -1344,6 +1257,7 @@ KLA_API kla_status_t kla_scan_forward_lti(const float *a, const void *phi, const
     kla::LtiParams prm;
     std::memset(&prm, 0, sizeof(prm));
     prm.a = a; prm.lam0 = lambda0; prm.eta0 = eta0;
+    prm.out[0] = lambda_out; prm.out[1] = eta_out; prm.out[2] = mu_out; prm.out[3] = var_out;
     prm.T = T; prm.HN = HN;
     prm.write_mu = mu_out != nullptr; prm.write_var = var_out != nullptr;
     prm.wait_ns = g_wait_ns.load();

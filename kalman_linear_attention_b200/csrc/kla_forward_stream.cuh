@@ -57,8 +57,13 @@ __device__ __forceinline__ void bulk_wait_group_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+#ifndef KLA_STREAM_DIRECT_STORE
+#define KLA_STREAM_DIRECT_STORE 0
+#endif
+
 struct StreamParams {
     const float *lam0, *eta0;      // [B, H, N] prior
+    float *out[4];                 // lambda, eta, mu, var [B, T, H, N] (mu / var may be null)
     int64_t T, HN;
     int64_t ntiles;                // B * ceil(HN / 32)
     int nct;                       // 32-channel tiles per batch row
@@ -329,6 +334,22 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             float lam, eta;
             chunk_carry(g, lam, eta);
             // (3) per-token recursion from the entering state
+#if KLA_STREAM_DIRECT_STORE
+            {
+                const int64_t base = (bb * prm.T + t0) * prm.HN + ch;
+#pragma unroll
+                for (int t = 0; t < L; ++t) {
+                    const TokenOut o = filter_token(lam, eta, xa[t], xp[t], xf[t], xb[t]);
+                    if (cvalid) {
+                        const int64_t i = base + (int64_t)t * prm.HN;
+                        __stcs(prm.out[0] + i, o.lam);
+                        __stcs(prm.out[1] + i, o.eta);
+                        if (prm.write_mu) __stcs(prm.out[2] + i, o.mu);
+                        if (prm.write_var) __stcs(prm.out[3] + i, o.var);
+                    }
+                }
+            }
+#else
 #pragma unroll
             for (int q = 0; q < L / G; ++q) {
                 float *buf = group_begin();
@@ -339,6 +360,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
                 }
                 group_end(buf, q);
             }
+#endif
         } else {
             // Ragged last chunk: straight from shared memory, released at the
             // end; rows past T are clipped by the TMA stores.

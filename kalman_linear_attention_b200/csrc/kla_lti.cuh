@@ -45,9 +45,14 @@
 
 namespace kla {
 
+#ifndef KLA_LTI_DIRECT_STORE
+#define KLA_LTI_DIRECT_STORE 0
+#endif
+
 struct LtiParams {
     const float *a;                // [B, H, N] time-invariant decay
     const float *lam0, *eta0;      // [B, H, N] prior
+    float *out[4];                 // lambda, eta, mu, var [B, T, H, N]; mu / var may be null
     int64_t T, HN;
     int64_t ntiles;                // B * ceil(HN / 32)
     int nct;                       // 32-channel tiles per batch row
@@ -302,6 +307,27 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
             sl = x[q * S + S - 1];
             se = y[q * S + S - 1];
         }
+#if KLA_LTI_DIRECT_STORE
+        // outputs straight from registers: one coalesced 128-byte row per
+        // output and token (rows past T and lanes past H*N are not stored)
+        if (cvalid) {
+            const int nv = (int)(prm.T - t0 < L ? prm.T - t0 : L);
+            const int64_t base = (bb * prm.T + t0) * prm.HN + ch;
+            float *o0 = prm.out[0] + base, *o1 = prm.out[1] + base;
+            float *o2 = prm.out[2] ? prm.out[2] + base : nullptr, *o3 = prm.out[3] ? prm.out[3] + base : nullptr;
+#pragma unroll
+            for (int t = 0; t < L; ++t) {
+                if (t < nv) {
+                    const float v = rcp_hw(x[t]);
+                    const int64_t off = (int64_t)t * prm.HN;
+                    __stcs(o0 + off, x[t]);
+                    __stcs(o1 + off, y[t]);
+                    if (o2) __stcs(o2 + off, y[t] * v);
+                    if (o3) __stcs(o3 + off, v);
+                }
+            }
+        }
+#else
 #pragma unroll
         for (int q = 0; q < L / G; ++q) {
             float *buf = outbuf0 + (group_seq & 1) * (Cfg::OUTBUF_BYTES / 4);
@@ -331,6 +357,7 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
             }
             ++group_seq;
         }
+#endif
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();

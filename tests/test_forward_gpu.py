@@ -17,11 +17,10 @@ def _kla():
     return kla
 
 
-@pytest.fixture(params=[1, 2, 3], ids=["chunked", "stream", "wide"])
+@pytest.fixture(params=[1, 2], ids=["chunked", "stream"])
 def kernel(request):
-    """Force one of the forward kernels (1: chunks exchange carries through
-    the workspace; 2: channel-owning streaming kernel; 3: one warp per 128
-    channels for the whole sequence -- 2 and 3 where their geometry holds)."""
+    """Force one of the two forward kernels (1: chunks exchange carries through
+    the workspace; 2: channel-owning streaming kernel, where its geometry holds)."""
     kla = _kla()
     kla.debug_force_forward_kernel(request.param)
     yield request.param
@@ -112,14 +111,13 @@ def test_kernels_agree_to_rounding():
     x = wl.generate(w)
     d = {k: torch.from_numpy(x[k]).to(DEV) for k in x}
     res = []
-    for which in (1, 2, 3):
+    for which in (1, 2):
         kla.debug_force_forward_kernel(which)
         assert kla.forward_plan(d["a"], d["p"], d["phi"], d["b"])[0] == which
         o = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
         res.append({k: t.double().cpu().numpy() for k, t in zip(parity.OUTPUTS, o)})
     kla.debug_force_forward_kernel(0)
     parity.assert_parity(res[1], res[0], 2e-6, time_axis=1, what="stream vs chunked")
-    parity.assert_parity(res[2], res[0], 2e-6, time_axis=1, what="wide vs chunked")
 
 
 def test_workspace_contents_do_not_matter(kernel):
@@ -226,12 +224,10 @@ def test_bitwise_reproducible(kernel):
 
 
 def test_plan_matches_workloads():
-    """On a B200: the tiny workload (2 tiles of 32 channels cannot occupy the
-    GPU) takes the chunked kernel, the long one (4096 channels) the streaming
-    kernel, and the LM-layer and stiff ones (1024 and 4096 channel tiles:
-    several warps per SM) the wide kernel."""
+    """On a B200 the standard workloads take the streaming kernel except the
+    tiny one (2 tiles of 32 channels cannot occupy the GPU)."""
     kla = _kla()
-    for name, expect in (("tiny", 1), ("lm_layer", 3), ("long", 2), ("stiff", 3)):
+    for name, expect in (("tiny", 1), ("lm_layer", 2), ("long", 2), ("stiff", 2)):
         w = wl.WORKLOADS[name]
         dt = parity.torch_dtype(w)
         z = torch.empty((w.B, w.T, w.H, w.N), dtype=dt, device=DEV)

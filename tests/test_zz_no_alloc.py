@@ -43,7 +43,7 @@ def _run(kla, w, force):
     x = wl.generate(w)
     dt = parity.torch_dtype(w)
     d = {k: torch.from_numpy(x[k]).to(DEV).to(dt) for k in wl.INPUT_NAMES}
-    pri = wl.random_prior(w)
+    pri = wl.prior(w)
     d["lam0"] = torch.from_numpy(pri["lam0"]).to(DEV)
     d["eta0"] = torch.from_numpy(pri["eta0"]).to(DEV)
     args = (d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
