@@ -111,7 +111,7 @@ class ClockSampler:
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,clocks.mem,clocks.max.mem")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -160,8 +160,11 @@ class ClockSampler:
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
         # under load: samples drawing more than the idle baseline
         loaded = [s for s, pw in zip(sm, power) if pw is not None and pw > 0.5 * max(power)] if power else sm
+        mem = [num(r[9]) for r in rows if len(r) > 9 and num(r[9]) is not None]
+        mem_max = [num(r[10]) for r in rows if len(r) > 10 and num(r[10]) is not None]
         return {"sm_mhz": statistics.median(loaded or sm), "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None,
+                "mem_mhz": statistics.median(mem) if mem else None, "mem_max_mhz": max(mem_max) if mem_max else None}
 
 
 # ----------------------------------------------------------------- our arm

@@ -487,8 +487,8 @@ kla_status_t kla_scan_forward_lti(const float *a, const void *phi, const void *b
 /*
  * Which kernel kla_scan_forward_lti would launch (only the alignment of phi
  * and b is looked at), written to *kernel: 1 = one thread per channel (any
- * shape), 2 = the channel-owning streaming kernel (16-byte aligned arrays,
- * H*N*elem a multiple of 16 bytes, H*N >= 32, T >= 32); *launches = kernel
+ * shape), 2 = the channel-owning streaming kernel (16-byte aligned phi and
+ * b, H*N*elem a multiple of 16 bytes, H*N >= 32, T >= 32); *launches = kernel
  * launches per call (2 when a workspace clear precedes the streaming
  * kernel).  0 and 0 for an empty problem.
  */

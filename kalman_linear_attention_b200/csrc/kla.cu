@@ -1165,17 +1165,13 @@ namespace {
 #ifndef KLA_LTI_S
 #define KLA_LTI_S 8
 #endif
-#ifndef KLA_LTI_G
-#define KLA_LTI_G 8
-#endif
 constexpr int kLtiL = 32;
-constexpr int kLtiG = KLA_LTI_G;
 
 template <typename Tin>
 constexpr int lti_stages() {
     constexpr int W = KLA_LTI_W;
     const int stage = 2 * kLtiL * 32 * (int)sizeof(Tin);
-    const int fixed = W * 2 * 4 * kLtiG * 32 * 4 + W * 2 * 32 * 8 + W * 8 + 2048;
+    const int fixed = W * 2 * 32 * 8 + W * 8 + 2048;
     const int ns = (KLA_STREAM_SMEM - fixed) / stage;
     return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
 }
@@ -1183,9 +1179,9 @@ constexpr int lti_stages() {
 template <typename Tin>
 cudaError_t launch_lti_stream(const kla::LtiParams &prm, const kla::LtiMaps &maps, cudaStream_t stream) {
     constexpr int NS = lti_stages<Tin>();
-    using Cfg = kla::LtiTile<Tin, kLtiL, KLA_LTI_W, NS, kLtiG>;
+    using Cfg = kla::LtiTile<Tin, kLtiL, KLA_LTI_W, NS>;
     static_assert(NS >= KLA_LTI_W && Cfg::SMEM <= 227 * 1024, "convolutional-form kernel shared memory");
-    auto kernel = kla::kla_lti_stream_kernel<Tin, kLtiL, KLA_LTI_S, KLA_LTI_W, NS, kLtiG>;
+    auto kernel = kla::kla_lti_stream_kernel<Tin, kLtiL, KLA_LTI_S, KLA_LTI_W, NS>;
     cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
@@ -1205,9 +1201,9 @@ StreamWs lti_ws_layout(int64_t ntiles, int parts) {
     return w;
 }
 
-// 2: the streaming kernel (TMA geometry as for the general streaming scan:
-// 16-byte aligned phi, b and outputs, H*N*elem a multiple of 16 bytes,
-// H*N >= 32, T >= 32); 1: one thread per channel (any shape).
+// 2: the streaming kernel (TMA loads as for the general streaming scan:
+// 16-byte aligned phi and b, H*N*elem a multiple of 16 bytes, H*N >= 32,
+// T >= 32); 1: one thread per channel (any shape).
 int lti_kernel_choice(int64_t T, int64_t HN, size_t esz, const void *const *ptrs, int n) {
     bool ok = (HN * (int64_t)esz) % 16 == 0 && T >= kLtiL && HN >= 32 && encode_fn() != nullptr;
     for (int k = 0; k < n && ok; ++k)
@@ -1263,17 +1259,13 @@ KLA_API kla_status_t kla_scan_forward_lti(const float *a, const void *phi, const
     prm.wait_ns = g_wait_ns.load();
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const void *ptrs[6] = {phi, b, lambda_out, eta_out, mu_out, var_out};
-    if (lti_kernel_choice(T, HN, esz, ptrs, 6) == 2) {
+    if (lti_kernel_choice(T, HN, esz, ptrs, 2) == 2) {  // phi and b: the outputs are stored without TMA
         const CUtensorMapDataType tdt =
             in_dtype == KLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
         kla::LtiMaps maps;
         std::memset(&maps, 0, sizeof(maps));
-        bool ok = encode_stream_map(&maps.in[0], phi, tdt, esz, B, T, HN, kLtiL) &&
-                  encode_stream_map(&maps.in[1], b, tdt, esz, B, T, HN, kLtiL);
-        float *outs4[4] = {lambda_out, eta_out, mu_out, var_out};
-        for (int k = 0; k < 4 && ok; ++k)
-            if (outs4[k]) ok = encode_stream_map(&maps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T,
-                                                 HN, kLtiG);
+        const bool ok = encode_stream_map(&maps.in[0], phi, tdt, esz, B, T, HN, kLtiL) &&
+                         encode_stream_map(&maps.in[1], b, tdt, esz, B, T, HN, kLtiL);
         if (ok) {
             prm.ntiles = B * ((HN + 31) / 32);
             prm.nct = (int)((HN + 31) / 32);

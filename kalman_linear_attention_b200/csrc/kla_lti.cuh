@@ -45,10 +45,6 @@
 
 namespace kla {
 
-#ifndef KLA_LTI_DIRECT_STORE
-#define KLA_LTI_DIRECT_STORE 0
-#endif
-
 struct LtiParams {
     const float *a;                // [B, H, N] time-invariant decay
     const float *lam0, *eta0;      // [B, H, N] prior
@@ -68,18 +64,14 @@ struct LtiParams {
 
 struct LtiMaps {
     CUtensorMap in[2];             // phi, b: {HN, T, B}, box {32, L, 1}
-    CUtensorMap out[4];            // lambda, eta, mu, var: box {32, G, 1}
 };
 
-template <typename Tin, int L, int W, int NS, int G>
+template <typename Tin, int L, int W, int NS>
 struct LtiTile {
     static_assert(NS >= W, "the stage ring must be at least as deep as the number of chunk warps");
-    static_assert(L % G == 0, "output groups must tile the chunk");
     static constexpr int THREADS = 32 * (W + 1);
     static constexpr int STAGE_BYTES = 2 * L * 32 * (int)sizeof(Tin);
-    static constexpr int OUTBUF_BYTES = 4 * G * 32 * 4;               // four outputs, one group
-    static constexpr int OUT_OFF = NS * STAGE_BYTES;                   // [W][2] output boxes
-    static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES;   // [W][2][32] fp64
+    static constexpr int CARRY_OFF = NS * STAGE_BYTES;                 // [W][2][32] fp64
     static constexpr int META_OFF = CARRY_OFF + W * 2 * 32 * 8;        // per stage: StreamChunk
     static constexpr int BAR_OFF = align_up(META_OFF + NS * (int)sizeof(StreamChunk), 128);
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
@@ -116,11 +108,11 @@ __device__ __forceinline__ void lti_powers(double a, LtiPowers<S, L> &w) {
     w.kL = nL * nL;
 }
 
-template <typename Tin, int L, int S, int W, int NS, int G>
+template <typename Tin, int L, int S, int W, int NS>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
 kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps) {
     static_assert(L % S == 0, "sub-blocks tile the chunk");
-    using Cfg = LtiTile<Tin, L, W, NS, G>;
+    using Cfg = LtiTile<Tin, L, W, NS>;
     constexpr int LC = L * 32;
     constexpr int NSB = L / S;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -198,8 +190,6 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
 
     // ------------------------------------------------------------ chunk warps
     const int w = warp - 1;
-    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
-    int group_seq = 0;
     int64_t power_tile = -1;  // tile whose kernel powers `kp` holds
     LtiPowers<S, L> kp;
 #pragma unroll 1
@@ -307,7 +297,6 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
             sl = x[q * S + S - 1];
             se = y[q * S + S - 1];
         }
-#if KLA_LTI_DIRECT_STORE
         // outputs straight from registers: one coalesced 128-byte row per
         // output and token (rows past T and lanes past H*N are not stored)
         if (cvalid) {
@@ -327,40 +316,7 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
                 }
             }
         }
-#else
-#pragma unroll
-        for (int q = 0; q < L / G; ++q) {
-            float *buf = outbuf0 + (group_seq & 1) * (Cfg::OUTBUF_BYTES / 4);
-            if (group_seq >= 2) {
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
-            }
-#pragma unroll
-            for (int u = 0; u < G; ++u) {
-                const int t = q * G + u;
-                const float v = rcp_hw(x[t]);
-                buf[u * 32 + lane] = x[t];
-                buf[G * 32 + u * 32 + lane] = y[t];
-                buf[2 * G * 32 + u * 32 + lane] = y[t] * v;
-                buf[3 * G * 32 + u * 32 + lane] = v;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                const int ty = (int)(t0 + q * G);
-                const int xo = (int)(ct * 32);
-                tma_store_3d(&maps.out[0], buf, xo, ty, (int)bb);
-                tma_store_3d(&maps.out[1], buf + G * 32, xo, ty, (int)bb);
-                if (prm.write_mu) tma_store_3d(&maps.out[2], buf + 2 * G * 32, xo, ty, (int)bb);
-                if (prm.write_var) tma_store_3d(&maps.out[3], buf + 3 * G * 32, xo, ty, (int)bb);
-                bulk_commit_group();
-            }
-            ++group_seq;
-        }
-#endif
     }
-    if (lane == 0) bulk_wait_group_all();
-    __syncwarp();
 }
 
 // Any shape (no TMA geometry needed): one thread per channel walks its
