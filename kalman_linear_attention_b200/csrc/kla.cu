@@ -96,13 +96,32 @@ template <typename Tin> constexpr int stream_warps() {
 template <typename Tin> constexpr int stream_group() {
     return sizeof(Tin) == 4 ? KLA_STREAM_G_F32 : KLA_STREAM_G_BF16;
 }
+// Two channels per lane (bf16 inputs with H*N >= 64): 64-channel tiles of
+// KLA_STREAM2_L-token chunks (the same registers per thread as 32 tokens x
+// one channel), chunk warps and output group.
+#ifndef KLA_STREAM2_L
+#define KLA_STREAM2_L 16
+#endif
+#ifndef KLA_STREAM2_W
+#define KLA_STREAM2_W 7
+#endif
+#ifndef KLA_STREAM2_G
+#define KLA_STREAM2_G 4
+#endif
+// 1 disables the two-channel layout (sweeps)
+#ifndef KLA_STREAM2_OFF
+#define KLA_STREAM2_OFF 0
+#endif
+
 // Ring stages that fit beside the per-warp output buffers and carry slots.
-template <typename Tin>
+template <typename Tin, int VEC = 1>
 constexpr int stream_stages() {
-    constexpr int W = stream_warps<Tin>();
-    constexpr int G = stream_group<Tin>();
-    const int stage = 4 * kSL * 32 * (int)sizeof(Tin);
-    const int fixed = W * 2 * 4 * G * 32 * 4 + W * 2 * 32 * 4 + W * 8 + 2048;
+    constexpr int W = VEC == 1 ? stream_warps<Tin>() : KLA_STREAM2_W;
+    constexpr int G = VEC == 1 ? stream_group<Tin>() : KLA_STREAM2_G;
+    constexpr int L = VEC == 1 ? kSL : KLA_STREAM2_L;
+    constexpr int CW = 32 * VEC;
+    const int stage = 4 * L * CW * (int)sizeof(Tin);
+    const int fixed = W * 2 * 4 * G * CW * 4 + W * 2 * CW * 4 + W * 8 + 2048;
     const int ns = (KLA_STREAM_SMEM - fixed) / stage;
     return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
 }
@@ -256,14 +275,15 @@ int sm_count() {
     return count[dev];
 }
 
-template <typename Tin>
+template <typename Tin, int VEC = 1>
 cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &maps, cudaStream_t stream) {
-    constexpr int W = stream_warps<Tin>();
-    constexpr int G = stream_group<Tin>();
-    constexpr int NS = stream_stages<Tin>();
-    using Cfg = kla::StreamTile<Tin, kSL, W, NS, G>;
+    constexpr int W = VEC == 1 ? stream_warps<Tin>() : KLA_STREAM2_W;
+    constexpr int G = VEC == 1 ? stream_group<Tin>() : KLA_STREAM2_G;
+    constexpr int L = VEC == 1 ? kSL : KLA_STREAM2_L;
+    constexpr int NS = stream_stages<Tin, VEC>();
+    using Cfg = kla::StreamTile<Tin, L, W, NS, G, VEC>;
     static_assert(NS >= 2 && Cfg::SMEM <= 227 * 1024, "stream kernel shared memory");
-    auto kernel = kla::kla_forward_stream_kernel<Tin, kSL, W, NS, G>;
+    auto kernel = kla::kla_forward_stream_kernel<Tin, L, W, NS, G, VEC>;
     cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
@@ -271,14 +291,14 @@ cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &m
     return cudaGetLastError();
 }
 
-// [B, T, HN] tensor viewed as dims {HN, T, B}, box {32, rows, 1}.
+// [B, T, HN] tensor viewed as dims {HN, T, B}, box {box_x, rows, 1}.
 bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, size_t esz,
-                       int64_t B, int64_t T, int64_t HN, int rows) {
+                       int64_t B, int64_t T, int64_t HN, int rows, int box_x = 32) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)HN, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[2] = {(cuuint64_t)(HN * esz), (cuuint64_t)(T * HN * esz)};
-    const cuuint32_t box[3] = {32u, (cuuint32_t)rows, 1u};
+    const cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)rows, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -293,9 +313,11 @@ bool encode_stream_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt,
 #ifndef KLA_STREAM_MAX_PARTS
 #define KLA_STREAM_MAX_PARTS 4
 #endif
-int stream_parts(int64_t ntiles, int64_t nchunks) {
+int stream_parts(int64_t ntiles, int64_t nchunks, int min_rounds = 2) {
+    // min_rounds: the fewest rounds of tiles (tiles / SMs) for which runs are
+    // cut; a run's predecessor is ticketed ntiles tickets before it
     const int64_t G = sm_count();
-    if (ntiles < 2 * G) return 1;
+    if (ntiles < min_rounds * G) return 1;
     int best = 1;
     double best_balance = 0.0;
     for (int P = 1; P <= KLA_STREAM_MAX_PARTS; ++P) {
@@ -317,14 +339,33 @@ int stream_parts(int64_t ntiles, int64_t nchunks) {
 struct StreamWs {
     size_t flags_off = 0, state_off = 0, clear_bytes = 0, total = 0;
 };
-StreamWs stream_ws_layout(int64_t ntiles, int parts) {
+StreamWs stream_ws_layout(int64_t ntiles, int parts, int cw = 32) {
     StreamWs w;
     const size_t nb = (size_t)ntiles * (size_t)(parts - 1);
     w.flags_off = kHeaderBytes;
     w.state_off = w.flags_off + round_up(nb * sizeof(unsigned), 256);
     w.clear_bytes = w.state_off;
-    w.total = w.state_off + round_up(nb * 64 * sizeof(float), 256);
+    w.total = w.state_off + round_up(nb * 2 * (size_t)cw * sizeof(float), 256);
     return w;
+}
+
+// The streaming forward kernel's layout for a call: two channels per lane
+// for bf16 inputs of at least 64 channels per batch row, else one.
+struct StreamGeom {
+    int vec, cw, L;
+    int64_t ntiles, nct, nchunks;
+    int parts;
+};
+StreamGeom stream_geom(int64_t B, int64_t T, int64_t HN, size_t esz) {
+    StreamGeom g;
+    g.vec = (esz == 2 && HN >= 64 && !KLA_STREAM2_OFF) ? 2 : 1;
+    g.cw = 32 * g.vec;
+    g.L = g.vec == 2 ? KLA_STREAM2_L : kSL;
+    g.nct = (HN + g.cw - 1) / g.cw;
+    g.ntiles = B * g.nct;
+    g.nchunks = (T + g.L - 1) / g.L;
+    g.parts = stream_parts(g.ntiles, g.nchunks, g.vec == 2 ? 1 : 2);
+    return g;
 }
 
 // 2: the channel-owning streaming kernel -- its TMA geometry holds (16-byte
@@ -387,8 +428,8 @@ KLA_API kla_status_t kla_scan_forward_workspace_size(int64_t B, int64_t T, int64
     }
     FwdLayout lay;
     if (!fwd_layout(B, T, HN, &lay)) return KLA_ERR_INVALID_ARG;
-    const int64_t ntiles32 = B * ((HN + 31) / 32);
-    const StreamWs sw = stream_ws_layout(ntiles32, KLA_STREAM_MAX_PARTS);  // the most runs stream_parts picks
+    const StreamGeom sg = stream_geom(B, T, HN, dtype_size(in_dtype));
+    const StreamWs sw = stream_ws_layout(sg.ntiles, KLA_STREAM_MAX_PARTS, sg.cw);  // the most runs stream_parts picks
     *bytes = std::max(lay.total, sw.total);
     return KLA_OK;
 }
@@ -454,41 +495,47 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
     // (it needs no workspace beyond its run splits); otherwise the chunked
     // kernel below.
     if (choice == 2) {
+        const StreamGeom sg = stream_geom(B, T, HN, esz);
+        const int G = sg.vec == 2 ? KLA_STREAM2_G
+                                  : (in_dtype == KLA_F32 ? stream_group<float>() : stream_group<__nv_bfloat16>());
         FwdMaps smaps;
         std::memset(&smaps, 0, sizeof(smaps));
         const void *ins4[4] = {a, p, phi, b};
         bool ok = true;
-        for (int k = 0; k < 4 && ok; ++k) ok = encode_stream_map(&smaps.in[k], ins4[k], tdt, esz, B, T, HN, kSL);
+        for (int k = 0; k < 4 && ok; ++k)
+            ok = encode_stream_map(&smaps.in[k], ins4[k], tdt, esz, B, T, HN, sg.L, sg.cw);
         float *outs4[4] = {lambda_out, eta_out, mu_out, var_out};
         for (int k = 0; k < 4 && ok; ++k)
             if (outs4[k])
-                ok = encode_stream_map(&smaps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN,
-                                       in_dtype == KLA_F32 ? stream_group<float>() : stream_group<__nv_bfloat16>());
+                ok = encode_stream_map(&smaps.out[k], outs4[k], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, HN, G, sg.cw);
         if (ok) {
             kla::StreamParams sp;
             sp.lam0 = lambda0; sp.eta0 = eta0;
-            sp.out[0] = lambda_out; sp.out[1] = eta_out; sp.out[2] = mu_out; sp.out[3] = var_out;
             sp.write_mu = mu_out != nullptr; sp.write_var = var_out != nullptr;
-            sp.T = T; sp.HN = HN; sp.ntiles = B * ((HN + 31) / 32);
-            sp.nct = (int)((HN + 31) / 32);
-            sp.nchunks = (int)((T + kSL - 1) / kSL);
+            sp.T = T; sp.HN = HN; sp.ntiles = sg.ntiles;
+            sp.nct = (int)sg.nct;
+            sp.nchunks = (int)sg.nchunks;
             sp.wait_ns = g_wait_ns.load();
-            sp.stall_chunk = g_stall_chunk.load() >= 0 ? g_stall_chunk.load() * kL / kSL : -1;
-            sp.parts = stream_parts(sp.ntiles, sp.nchunks);
+            sp.stall_chunk = g_stall_chunk.load() >= 0 ? g_stall_chunk.load() * kL / sg.L : -1;
+            sp.parts = sg.parts;
             sp.chunks_per_part = (sp.nchunks + sp.parts - 1) / sp.parts;
             sp.nunits = sp.ntiles * sp.parts;
             sp.ticket = reinterpret_cast<unsigned *>(ws);
             sp.part_flags = nullptr;
             sp.part_state = nullptr;
             if (sp.parts > 1) {
-                const StreamWs sw = stream_ws_layout(sp.ntiles, sp.parts);
+                const StreamWs sw = stream_ws_layout(sp.ntiles, sp.parts, sg.cw);
                 if (sw.total > workspace_bytes) return KLA_ERR_WORKSPACE_TOO_SMALL;  // size function out of step
                 sp.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
                 sp.part_state = reinterpret_cast<float *>(ws + sw.state_off);
                 if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
             }
-            const cudaError_t es = in_dtype == KLA_F32 ? launch_forward_stream<float>(sp, smaps, st)
-                                                       : launch_forward_stream<__nv_bfloat16>(sp, smaps, st);
+            cudaError_t es;
+            if (in_dtype == KLA_F32)
+                es = launch_forward_stream<float>(sp, smaps, st);
+            else
+                es = sg.vec == 2 ? launch_forward_stream<__nv_bfloat16, 2>(sp, smaps, st)
+                                 : launch_forward_stream<__nv_bfloat16>(sp, smaps, st);
             return es == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
         }
     }
@@ -617,8 +664,7 @@ KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int6
     *kernel = forward_kernel_choice(B, T, HN, dtype_size(in_dtype), a, p, phi, b, nullptr, nullptr, nullptr,
                                     nullptr);
     *launches = 2;  // chunked kernel: workspace clear + scan
-    if (*kernel == 2)
-        *launches = stream_parts(B * ((HN + 31) / 32), (T + kSL - 1) / kSL) > 1 ? 2 : 1;
+    if (*kernel == 2) *launches = stream_geom(B, T, HN, dtype_size(in_dtype)).parts > 1 ? 2 : 1;
     return KLA_OK;
 }
 

@@ -26,6 +26,11 @@
 //                   also clip ragged edges), so the chunk warps do no global
 //                   address arithmetic.
 //
+// A lane owns VEC consecutive channels (CW = 32 VEC per tile): with VEC = 2
+// (bf16 inputs: 64-channel tiles, 16-token chunks, the same registers per
+// thread) every lane runs two independent recursion chains side by side, and
+// one 32-bit shared load brings a token's two bf16 values of an input.
+//
 // Within a tile no global flags, fences or look-back: the W warps overlap
 // their passes while the producer keeps HBM busy.  Chunk aggregates are formed
 // and applied exactly as in kla_forward_kernel (one thread's run = the whole
@@ -57,16 +62,11 @@ __device__ __forceinline__ void bulk_wait_group_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-#ifndef KLA_STREAM_DIRECT_STORE
-#define KLA_STREAM_DIRECT_STORE 0
-#endif
-
 struct StreamParams {
     const float *lam0, *eta0;      // [B, H, N] prior
-    float *out[4];                 // lambda, eta, mu, var [B, T, H, N] (mu / var may be null)
     int64_t T, HN;
-    int64_t ntiles;                // B * ceil(HN / 32)
-    int nct;                       // 32-channel tiles per batch row
+    int64_t ntiles;                // B * ceil(HN / CW)
+    int nct;                       // tiles of CW channels per batch row
     int nchunks;                   // ceil(T / L)
     int write_mu, write_var;       // outputs 2 / 3 requested
     uint64_t wait_ns;
@@ -79,7 +79,7 @@ struct StreamParams {
     int64_t nunits;                // ntiles * parts
     unsigned *ticket;              // parts > 1: unit counter (zeroed per call)
     unsigned *part_flags;          // [ntiles][parts - 1], zeroed per call
-    float *part_state;             // [ntiles][parts - 1][2][32]
+    float *part_state;             // [ntiles][parts - 1][2][CW]
     int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
 };
 
@@ -93,7 +93,7 @@ struct StreamChunk {
     int first, last;               // chunks of the run
 };
 
-template <typename Tin, int L, int W, int NS, int G>
+template <typename Tin, int L, int W, int NS, int G, int VEC = 1>
 struct StreamTile {
     // Chunk j sits in stage j % NS and is handled by warp j % W.  With
     // NS >= W a warp waiting for stage s is always waiting for the stage's
@@ -102,13 +102,14 @@ struct StreamTile {
     // unambiguous.  With NS < W a warp could pass a wait one phase early.
     static_assert(NS >= W, "the stage ring must be at least as deep as the number of chunk warps");
     static_assert(L % G == 0, "output groups must tile the chunk");
-    static constexpr int CW = 32;
+    static_assert(VEC == 1 || VEC == 2, "one or two channels per lane");
+    static constexpr int CW = 32 * VEC;                              // channels per tile
     static constexpr int THREADS = 32 * (W + 1);                     // producer + W chunk warps
     static constexpr int STAGE_BYTES = 4 * L * CW * (int)sizeof(Tin);
     static constexpr int OUTBOX_BYTES = G * CW * 4;                 // one output, one group
     static constexpr int OUTBUF_BYTES = 4 * OUTBOX_BYTES;           // four outputs
-    static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][32] fp32
-    static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][32] fp32
+    static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][CW] fp32
+    static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][CW] fp32
     static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: unit (int64), chunk (int64)
     static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128); // full, empty, carry
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
@@ -121,11 +122,38 @@ __device__ __forceinline__ void mbar_wait_or_flag(uint64_t *bar, unsigned parity
     }
 }
 
-template <typename Tin, int L, int W, int NS, int G>
+// The VEC consecutive values of a lane in one row of a stage (CW = 32 VEC
+// values of one input and token), widened to fp32.
+template <typename Tin, int VEC> struct RowVec;
+template <typename Tin> struct RowVec<Tin, 1> {
+    static __device__ __forceinline__ void load(const Tin *row, int lane, float (&v)[1]) { v[0] = to_f32(row[lane]); }
+};
+template <> struct RowVec<float, 2> {
+    static __device__ __forceinline__ void load(const float *row, int lane, float (&v)[2]) {
+        const float2 x = reinterpret_cast<const float2 *>(row)[lane];
+        v[0] = x.x; v[1] = x.y;
+    }
+};
+template <> struct RowVec<__nv_bfloat16, 2> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *row, int lane, float (&v)[2]) {
+        const unsigned u = reinterpret_cast<const unsigned *>(row)[lane];  // channel 2 lane in the low half
+        v[0] = __uint_as_float(u << 16);
+        v[1] = __uint_as_float(u & 0xffff0000u);
+    }
+};
+
+// VEC consecutive floats into shared memory.
+__device__ __forceinline__ void sts_vec(float *dst, const float (&v)[1]) { *dst = v[0]; }
+__device__ __forceinline__ void sts_vec(float *dst, const float (&v)[2]) {
+    *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
+}
+
+template <typename Tin, int L, int W, int NS, int G, int VEC = 1>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
 kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMaps maps) {
-    using Cfg = StreamTile<Tin, L, W, NS, G>;
-    constexpr int LC = L * 32;
+    using Cfg = StreamTile<Tin, L, W, NS, G, VEC>;
+    constexpr int CW = Cfg::CW;
+    constexpr int LC = L * CW;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::BAR_OFF);
     uint64_t *empty = full + NS;
@@ -169,7 +197,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, chunk * L, bb, &full[s]);
+                tma_load_3d(stage + q * LC, &maps.in[q], ct * CW, chunk * L, bb, &full[s]);
         };
         // one unit: the tile's run u / ntiles, in time order (its tile
         // coordinates computed once per unit, not per chunk)
@@ -208,6 +236,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
     const int w = warp - 1;
     float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
     int group_seq = 0;  // output groups this warp has committed (bulk groups are per thread: lane 0)
+    const int lc = lane * VEC;  // this lane's first channel within a tile
 #pragma unroll 1
     for (int64_t j = w;; j += W) {
         const int s = (int)(j % NS);
@@ -221,8 +250,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
         const int64_t ct = tile - bb * prm.nct;
         const int64_t t0 = chunk * L;
         const int t_valid = (int)(prm.T - t0 < (int64_t)L ? prm.T - t0 : (int64_t)L);
-        const int64_t ch = ct * 32 + lane;
-        const bool cvalid = ch < prm.HN;
+        const int64_t ch = ct * CW + lc;  // the lane's channels ch .. ch + VEC - 1
         const Tin *stage = reinterpret_cast<const Tin *>(smem + s * Cfg::STAGE_BYTES);
         const int64_t first = part * prm.chunks_per_part;  // first chunk of this unit
         const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
@@ -232,43 +260,67 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
         // prior at a tile's first chunk, or from the previous run of the tile
         // at a later run's first chunk -- and the state leaving it, handed to
         // the next warp (and published for the next run at a run's end).
-        auto chunk_carry = [&](const Agg &g, float &lam, float &eta) {
+        auto chunk_carry = [&](const Agg (&g)[VEC], float (&lam)[VEC], float (&eta)[VEC]) {
             if (j > 0) {
                 const int ps = (int)((j - 1) % W);
                 mbar_wait_or_flag(&carry_bar[ps], (unsigned)(((j - 1) / W) & 1), prm.wait_ns);
-                lam = slots[ps * 64 + lane];
-                eta = slots[ps * 64 + 32 + lane];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    lam[v] = slots[ps * 2 * CW + lc + v];
+                    eta[v] = slots[ps * 2 * CW + CW + lc + v];
+                }
             }
             if (chunk == prm.stall_chunk &&
                 !warp_wait_flags(lane == 0 ? &g_never_set_word : nullptr, prm.wait_ns)) {
-                lam = __int_as_float(0x7fc00000);  // ran out of time: poison what follows
-                eta = lam;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    lam[v] = __int_as_float(0x7fc00000);  // ran out of time: poison what follows
+                    eta[v] = lam[v];
+                }
                 if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
             } else if (chunk == 0) {
-                lam = cvalid ? prm.lam0[bb * prm.HN + ch] : 1.f;
-                eta = cvalid ? prm.eta0[bb * prm.HN + ch] : 0.f;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    const bool cvalid = ch + v < prm.HN;
+                    lam[v] = cvalid ? prm.lam0[bb * prm.HN + ch + v] : 1.f;
+                    eta[v] = cvalid ? prm.eta0[bb * prm.HN + ch + v] : 0.f;
+                }
             } else if (chunk == first) {
                 const int64_t slot = tile * (prm.parts - 1) + (part - 1);
                 if (warp_wait_flags(lane == 0 ? prm.part_flags + slot : nullptr, prm.wait_ns)) {
-                    lam = __ldcg(prm.part_state + slot * 64 + lane);
-                    eta = __ldcg(prm.part_state + slot * 64 + 32 + lane);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        lam[v] = __ldcg(prm.part_state + slot * 2 * CW + lc + v);
+                        eta[v] = __ldcg(prm.part_state + slot * 2 * CW + CW + lc + v);
+                    }
                 } else {
-                    lam = __int_as_float(0x7fc00000);
-                    eta = lam;
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        lam[v] = __int_as_float(0x7fc00000);
+                        eta[v] = lam[v];
+                    }
                     if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
                 }
             }
-            float lo = lam, eo = eta;
-            agg_apply(g, lo, eo);
+            float lo[VEC], eo[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                lo[v] = lam[v];
+                eo[v] = eta[v];
+                agg_apply(g[v], lo[v], eo[v]);
+            }
             const int ms = (int)(j % W);
-            slots[ms * 64 + lane] = lo;
-            slots[ms * 64 + 32 + lane] = eo;
+            sts_vec(slots + ms * 2 * CW + lc, lo);
+            sts_vec(slots + ms * 2 * CW + CW + lc, eo);
             __syncwarp();
             if (lane == 0) mbar_arrive(&carry_bar[ms]);
             if (chunk == last && part + 1 < prm.parts) {
                 const int64_t slot = tile * (prm.parts - 1) + part;
-                prm.part_state[slot * 64 + lane] = lo;
-                prm.part_state[slot * 64 + 32 + lane] = eo;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    prm.part_state[slot * 2 * CW + lc + v] = lo[v];
+                    prm.part_state[slot * 2 * CW + CW + lc + v] = eo[v];
+                }
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) st_release_gpu(prm.part_flags + slot, 1u);
@@ -291,89 +343,94 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             __syncwarp();
             if (lane == 0) {
                 const int ty = (int)(t0 + q * G);
-                const int x = (int)(ct * 32);
+                const int x = (int)(ct * CW);
                 tma_store_3d(&maps.out[0], buf, x, ty, (int)bb);
-                tma_store_3d(&maps.out[1], buf + G * 32, x, ty, (int)bb);
-                if (prm.write_mu) tma_store_3d(&maps.out[2], buf + 2 * G * 32, x, ty, (int)bb);
-                if (prm.write_var) tma_store_3d(&maps.out[3], buf + 3 * G * 32, x, ty, (int)bb);
+                tma_store_3d(&maps.out[1], buf + G * CW, x, ty, (int)bb);
+                if (prm.write_mu) tma_store_3d(&maps.out[2], buf + 2 * G * CW, x, ty, (int)bb);
+                if (prm.write_var) tma_store_3d(&maps.out[3], buf + 3 * G * CW, x, ty, (int)bb);
                 bulk_commit_group();
             }
             ++group_seq;
         };
-        auto put = [&](float *buf, int u, const TokenOut &o) {
-            buf[u * 32 + lane] = o.lam;
-            buf[G * 32 + u * 32 + lane] = o.eta;
-            buf[2 * G * 32 + u * 32 + lane] = o.mu;
-            buf[3 * G * 32 + u * 32 + lane] = o.var;
+        // token u of the group: the four outputs of the lane's VEC channels
+        auto run_token = [&](float *buf, int u, float (&lam)[VEC], float (&eta)[VEC], const float (&a)[VEC],
+                             const float (&p)[VEC], const float (&f)[VEC], const float (&b)[VEC]) {
+            float ol[VEC], oe[VEC], om[VEC], ov[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                const TokenOut o = filter_token(lam[v], eta[v], a[v], p[v], f[v], b[v]);
+                ol[v] = o.lam; oe[v] = o.eta; om[v] = o.mu; ov[v] = o.var;
+            }
+            sts_vec(buf + u * CW + lc, ol);
+            sts_vec(buf + G * CW + u * CW + lc, oe);
+            sts_vec(buf + 2 * G * CW + u * CW + lc, om);
+            sts_vec(buf + 3 * G * CW + u * CW + lc, ov);
         };
 
         if (t_valid == L) {
             // Full chunk: read it from shared memory once into registers,
             // release the stage to the producer right away, then run both
             // passes from registers.
-            float xa[L], xp[L], xf[L], xb[L];
+            float xa[L][VEC], xp[L][VEC], xf[L][VEC], xb[L][VEC];
 #pragma unroll
             for (int t = 0; t < L; ++t) {
-                const int i = t * 32 + lane;
-                xa[t] = to_f32(stage[i]);
-                xp[t] = to_f32(stage[LC + i]);
-                xf[t] = to_f32(stage[2 * LC + i]);
-                xb[t] = to_f32(stage[3 * LC + i]);
+                RowVec<Tin, VEC>::load(stage + t * CW, lane, xa[t]);
+                RowVec<Tin, VEC>::load(stage + LC + t * CW, lane, xp[t]);
+                RowVec<Tin, VEC>::load(stage + 2 * LC + t * CW, lane, xf[t]);
+                RowVec<Tin, VEC>::load(stage + 3 * LC + t * CW, lane, xb[t]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
-            // (1) the chunk's aggregate (renormalised every second token)
-            Agg g = agg_identity();
+            // (1) the chunk's aggregates (renormalised every second token)
+            Agg g[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) g[v] = agg_identity();
 #pragma unroll
             for (int t = 0; t < L; ++t) {
-                agg_push_token(g, xa[t], xp[t], xf[t], xb[t]);
-                if (renorm_after(t)) agg_renorm(g);
-            }
-            agg_renorm(g);
-            // (2) carry
-            float lam, eta;
-            chunk_carry(g, lam, eta);
-            // (3) per-token recursion from the entering state
-#if KLA_STREAM_DIRECT_STORE
-            {
-                const int64_t base = (bb * prm.T + t0) * prm.HN + ch;
 #pragma unroll
-                for (int t = 0; t < L; ++t) {
-                    const TokenOut o = filter_token(lam, eta, xa[t], xp[t], xf[t], xb[t]);
-                    if (cvalid) {
-                        const int64_t i = base + (int64_t)t * prm.HN;
-                        __stcs(prm.out[0] + i, o.lam);
-                        __stcs(prm.out[1] + i, o.eta);
-                        if (prm.write_mu) __stcs(prm.out[2] + i, o.mu);
-                        if (prm.write_var) __stcs(prm.out[3] + i, o.var);
-                    }
+                for (int v = 0; v < VEC; ++v) {
+                    agg_push_token(g[v], xa[t][v], xp[t][v], xf[t][v], xb[t][v]);
+                    if (renorm_after(t)) agg_renorm(g[v]);
                 }
             }
-#else
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) agg_renorm(g[v]);
+            // (2) carry
+            float lam[VEC], eta[VEC];
+            chunk_carry(g, lam, eta);
+            // (3) per-token recursion from the entering state
 #pragma unroll
             for (int q = 0; q < L / G; ++q) {
                 float *buf = group_begin();
 #pragma unroll
                 for (int u = 0; u < G; ++u) {
                     const int t = q * G + u;
-                    put(buf, u, filter_token(lam, eta, xa[t], xp[t], xf[t], xb[t]));
+                    run_token(buf, u, lam, eta, xa[t], xp[t], xf[t], xb[t]);
                 }
                 group_end(buf, q);
             }
-#endif
         } else {
             // Ragged last chunk: straight from shared memory, released at the
             // end; rows past T are clipped by the TMA stores.
-            Agg g = agg_identity();
+            Agg g[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) g[v] = agg_identity();
 #pragma unroll 2
             for (int t = 0; t < t_valid; ++t) {
-                const int i = t * 32 + lane;
-                agg_push_token(g, to_f32(stage[i]), to_f32(stage[LC + i]), to_f32(stage[2 * LC + i]),
-                               to_f32(stage[3 * LC + i]));
-                if (renorm_after(t)) agg_renorm(g);
+                float a[VEC], p[VEC], f[VEC], b[VEC];
+                RowVec<Tin, VEC>::load(stage + t * CW, lane, a);
+                RowVec<Tin, VEC>::load(stage + LC + t * CW, lane, p);
+                RowVec<Tin, VEC>::load(stage + 2 * LC + t * CW, lane, f);
+                RowVec<Tin, VEC>::load(stage + 3 * LC + t * CW, lane, b);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    agg_push_token(g[v], a[v], p[v], f[v], b[v]);
+                    if (renorm_after(t)) agg_renorm(g[v]);
+                }
             }
-            agg_renorm(g);
-            float lam, eta;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) agg_renorm(g[v]);
+            float lam[VEC], eta[VEC];
             chunk_carry(g, lam, eta);
             const int ngroups = (t_valid + G - 1) / G;
 #pragma unroll 1
@@ -383,9 +440,12 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
                 for (int u = 0; u < G; ++u) {
                     const int t = q * G + u;
                     if (t < t_valid) {
-                        const int i = t * 32 + lane;
-                        put(buf, u, filter_token(lam, eta, to_f32(stage[i]), to_f32(stage[LC + i]),
-                                                 to_f32(stage[2 * LC + i]), to_f32(stage[3 * LC + i])));
+                        float a[VEC], p[VEC], f[VEC], b[VEC];
+                        RowVec<Tin, VEC>::load(stage + t * CW, lane, a);
+                        RowVec<Tin, VEC>::load(stage + LC + t * CW, lane, p);
+                        RowVec<Tin, VEC>::load(stage + 2 * LC + t * CW, lane, f);
+                        RowVec<Tin, VEC>::load(stage + 3 * LC + t * CW, lane, b);
+                        run_token(buf, u, lam, eta, a, p, f, b);
                     }
                 }
                 group_end(buf, q);
