@@ -70,19 +70,29 @@ __global__ void __launch_bounds__(256) kla_attention_kernel(const AttnParams prm
     const Tin *pg = static_cast<const Tin *>(prm.p);
 
     // 1) the gate of every window token after the first (the first one's is
-    //    never used: F(t, s) takes the gates of tokens s+1..t)
-    for (int idx = threadIdx.x; idx < nv * CW; idx += blockDim.x) {
-        const int k = idx / CW;
-        const int c = idx - k * CW;
-        float g = 0.f;
-        if (k >= 1 && c0 + c < prm.HN) {
-            const int64_t row = (bb * prm.T + start + k) * prm.HN + c0 + c;
-            const float a = to_f32(ag[row]);
-            const float p = to_f32(pg[row]);
-            const float lam_before = __ldg(prm.lam + row - prm.HN);  // lambda_{k-1}: this channel, previous token
-            g = a * rcp_hw(fmaf(p, lam_before, a * a));
+    //    never used: F(t, s) takes the gates of tokens s+1..t); each thread
+    //    issues the loads of GU elements before their arithmetic
+    constexpr int GU = 8;
+    for (int base = threadIdx.x; base < nv * CW; base += GU * blockDim.x) {
+        float av[GU], pv[GU], lv[GU];
+#pragma unroll
+        for (int u = 0; u < GU; ++u) {
+            const int idx = base + u * blockDim.x;
+            const int k = idx / CW;
+            const int c = idx - k * CW;
+            av[u] = 0.f; pv[u] = 1.f; lv[u] = 1.f;  // an unused gate: 0
+            if (idx < nv * CW && k >= 1 && c0 + c < prm.HN) {
+                const int64_t row = (bb * prm.T + start + k) * prm.HN + c0 + c;
+                av[u] = to_f32(ag[row]);
+                pv[u] = to_f32(pg[row]);
+                lv[u] = __ldg(prm.lam + row - prm.HN);  // lambda_{k-1}: this channel, previous token
+            }
         }
-        gates[idx] = g;
+#pragma unroll
+        for (int u = 0; u < GU; ++u) {
+            const int idx = base + u * blockDim.x;
+            if (idx < nv * CW) gates[idx] = av[u] * rcp_hw(fmaf(pv[u], lv[u], av[u] * av[u]));
+        }
     }
     __syncthreads();
 
@@ -95,28 +105,34 @@ __global__ void __launch_bounds__(256) kla_attention_kernel(const AttnParams prm
     const int64_t WW = (int64_t)prm.W * prm.W;
     float *Fcta = prm.F + ((bb * prm.nwin + win) * WW) * prm.HN + c0 + lane * VEC;
     const float *glane = gates + lane * VEC;
+    const int64_t row_step = (int64_t)prm.W * prm.HN;  // elements from row i to row i + 1 of a column
 #pragma unroll 1
     for (int j = warp; j < prm.W; j += nwarps) {
+        if (!cvalid) continue;
         float f[VEC];
 #pragma unroll
         for (int v = 0; v < VEC; ++v) f[v] = 1.f;
-        float *col = Fcta + (int64_t)j * prm.HN;
         const float zero[VEC] = {};
-#pragma unroll 1
-        for (int i = 0; i < prm.W; ++i) {
-            float *dst = col + (int64_t)i * prm.W * prm.HN;
-            if (i < j || i >= nv || j >= nv) {
-                if (cvalid) st_cs_vec(dst, zero);
-            } else {
-                if (i > j) {
-                    float g[VEC];
-                    lds_vec(g, glane + i * CW);
+        float *dst = Fcta + (int64_t)j * prm.HN;
+        // rows above the diagonal (and the whole column past the span): zeros
+        const int lo = j < nv ? j : prm.W;
+#pragma unroll 4
+        for (int i = 0; i < lo; ++i, dst += row_step) st_cs_vec(dst, zero);
+        if (j >= nv) continue;
+        // the diagonal, then the running product of the gates down the column
+        st_cs_vec(dst, f);
+        dst += row_step;
+#pragma unroll 4
+        for (int i = j + 1; i < nv; ++i, dst += row_step) {
+            float g[VEC];
+            lds_vec(g, glane + i * CW);
 #pragma unroll
-                    for (int v = 0; v < VEC; ++v) f[v] *= g[v];
-                }
-                if (cvalid) st_cs_vec(dst, f);
-            }
+            for (int v = 0; v < VEC; ++v) f[v] *= g[v];
+            st_cs_vec(dst, f);
         }
+        // rows past the span
+#pragma unroll 4
+        for (int i = nv; i < prm.W; ++i, dst += row_step) st_cs_vec(dst, zero);
     }
 }
 

@@ -302,18 +302,27 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
         if (cvalid) {
             const int nv = (int)(prm.T - t0 < L ? prm.T - t0 : L);
             const int64_t base = (bb * prm.T + t0) * prm.HN + ch;
+            const int64_t hn = prm.HN;
             float *o0 = prm.out[0] + base, *o1 = prm.out[1] + base;
-            float *o2 = prm.out[2] ? prm.out[2] + base : nullptr, *o3 = prm.out[3] ? prm.out[3] + base : nullptr;
+            float *o2 = prm.write_mu ? prm.out[2] + base : nullptr;
+            float *o3 = prm.write_var ? prm.out[3] + base : nullptr;
+            auto put = [&](int t) {
+                const float v = rcp_hw(x[t]);
+                __stcs(o0, x[t]);
+                __stcs(o1, y[t]);
+                if (o2) __stcs(o2, y[t] * v);
+                if (o3) __stcs(o3, v);
+                o0 += hn; o1 += hn;
+                if (o2) o2 += hn;
+                if (o3) o3 += hn;
+            };
+            if (nv == L) {
 #pragma unroll
-            for (int t = 0; t < L; ++t) {
-                if (t < nv) {
-                    const float v = rcp_hw(x[t]);
-                    const int64_t off = (int64_t)t * prm.HN;
-                    __stcs(o0 + off, x[t]);
-                    __stcs(o1 + off, y[t]);
-                    if (o2) __stcs(o2 + off, y[t] * v);
-                    if (o3) __stcs(o3 + off, v);
-                }
+                for (int t = 0; t < L; ++t) put(t);
+            } else {
+#pragma unroll
+                for (int t = 0; t < L; ++t)
+                    if (t < nv) put(t);
             }
         }
     }
