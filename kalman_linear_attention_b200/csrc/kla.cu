@@ -98,7 +98,9 @@ template <typename Tin> constexpr int stream_group() {
 }
 // Two channels per lane (bf16 inputs with H*N >= 64): 64-channel tiles of
 // KLA_STREAM2_L-token chunks (the same registers per thread as 32 tokens x
-// one channel), chunk warps and output group.
+// one channel), chunk warps and output group.  On the LM-layer shape: 5%
+// faster than one channel per lane with 8-token output groups, no faster
+// with 4, slower with 6 chunk warps.
 #ifndef KLA_STREAM2_L
 #define KLA_STREAM2_L 16
 #endif
@@ -106,7 +108,7 @@ template <typename Tin> constexpr int stream_group() {
 #define KLA_STREAM2_W 7
 #endif
 #ifndef KLA_STREAM2_G
-#define KLA_STREAM2_G 4
+#define KLA_STREAM2_G 8
 #endif
 // 1 disables the two-channel layout (sweeps)
 #ifndef KLA_STREAM2_OFF
@@ -283,11 +285,18 @@ cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &m
     constexpr int NS = stream_stages<Tin, VEC>();
     using Cfg = kla::StreamTile<Tin, L, W, NS, G, VEC>;
     static_assert(NS >= 2 && Cfg::SMEM <= 227 * 1024, "stream kernel shared memory");
-    auto kernel = kla::kla_forward_stream_kernel<Tin, L, W, NS, G, VEC>;
-    cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(prm.nunits, sm_count());
-    kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    if constexpr (VEC == 1) {
+        auto kernel = kla::kla_forward_stream_kernel<Tin, L, W, NS, G>;
+        cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    } else {
+        auto kernel = kla::kla_forward_stream_vec_kernel<Tin, L, W, NS, G, VEC>;
+        cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+    }
     return cudaGetLastError();
 }
 

@@ -148,9 +148,274 @@ __device__ __forceinline__ void sts_vec(float *dst, const float (&v)[2]) {
     *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
 }
 
-template <typename Tin, int L, int W, int NS, int G, int VEC = 1>
+template <typename Tin, int L, int W, int NS, int G>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
 kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMaps maps) {
+    using Cfg = StreamTile<Tin, L, W, NS, G>;
+    constexpr int LC = L * 32;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::BAR_OFF);
+    uint64_t *empty = full + NS;
+    uint64_t *carry_bar = empty + NS;
+    float *slots = reinterpret_cast<float *>(smem + Cfg::CARRY_OFF);
+    int64_t *meta_unit = reinterpret_cast<int64_t *>(smem + Cfg::META_OFF);  // -1: no more work
+    int64_t *meta_chunk = meta_unit + NS;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < W; ++s) mbar_init(&carry_bar[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane != 0) return;
+        int next = 0, round = 0;  // next stage to fill; completed passes over the ring
+        auto claim = [&]() -> int {
+            const int s = next;
+            if (round > 0) mbar_wait_or_flag(&empty[s], (unsigned)((round - 1) & 1), prm.wait_ns);
+            if (++next == NS) {
+                next = 0;
+                ++round;
+            }
+            return s;
+        };
+        auto load = [&](int64_t unit, int chunk, int bb, int ct) {
+            const int s = claim();
+            meta_unit[s] = unit;
+            meta_chunk[s] = chunk;
+            Tin *stage = reinterpret_cast<Tin *>(smem + s * Cfg::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full[s], (unsigned)Cfg::STAGE_BYTES);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                tma_load_3d(stage + q * LC, &maps.in[q], ct * 32, chunk * L, bb, &full[s]);
+        };
+        // one unit: the tile's run u / ntiles, in time order (its tile
+        // coordinates computed once per unit, not per chunk)
+        auto unit_chunks = [&](int64_t u) {
+            const int64_t tile = u % prm.ntiles;
+            const int part = (int)(u / prm.ntiles);
+            const int bb = (int)(tile / prm.nct);
+            const int ct = (int)(tile - (int64_t)bb * prm.nct);
+            const int first = part * prm.chunks_per_part;
+            const int last = min(first + prm.chunks_per_part, prm.nchunks) - 1;
+#pragma unroll 1
+            for (int c = first; c <= last; ++c) load(u, c, bb, ct);
+        };
+        if (prm.parts == 1) {
+#pragma unroll 1
+            for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
+        } else {
+#pragma unroll 1
+            for (;;) {
+                const int64_t u = (int64_t)atomicAdd(prm.ticket, 1u);
+                if (u >= prm.nunits) break;
+                unit_chunks(u);
+            }
+        }
+        // one end marker for each chunk warp
+#pragma unroll 1
+        for (int k = 0; k < W; ++k) {
+            const int s = claim();
+            meta_unit[s] = -1;
+            mbar_arrive(&full[s]);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------ chunk warps
+    const int w = warp - 1;
+    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
+    int group_seq = 0;  // output groups this warp has committed (bulk groups are per thread: lane 0)
+#pragma unroll 1
+    for (int64_t j = w;; j += W) {
+        const int s = (int)(j % NS);
+        mbar_wait_or_flag(&full[s], (unsigned)((j / NS) & 1), prm.wait_ns);
+        const int64_t unit = meta_unit[s];
+        if (unit < 0) break;
+        const int64_t chunk = meta_chunk[s];
+        const int64_t tile = unit % prm.ntiles;
+        const int64_t part = unit / prm.ntiles;
+        const int64_t bb = tile / prm.nct;
+        const int64_t ct = tile - bb * prm.nct;
+        const int64_t t0 = chunk * L;
+        const int t_valid = (int)(prm.T - t0 < (int64_t)L ? prm.T - t0 : (int64_t)L);
+        const int64_t ch = ct * 32 + lane;
+        const bool cvalid = ch < prm.HN;
+        const Tin *stage = reinterpret_cast<const Tin *>(smem + s * Cfg::STAGE_BYTES);
+        const int64_t first = part * prm.chunks_per_part;  // first chunk of this unit
+        const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
+                                                                         : (int64_t)prm.nchunks) - 1;
+
+        // State entering chunk j -- from the previous chunk's warp, from the
+        // prior at a tile's first chunk, or from the previous run of the tile
+        // at a later run's first chunk -- and the state leaving it, handed to
+        // the next warp (and published for the next run at a run's end).
+        auto chunk_carry = [&](const Agg &g, float &lam, float &eta) {
+            if (j > 0) {
+                const int ps = (int)((j - 1) % W);
+                mbar_wait_or_flag(&carry_bar[ps], (unsigned)(((j - 1) / W) & 1), prm.wait_ns);
+                lam = slots[ps * 64 + lane];
+                eta = slots[ps * 64 + 32 + lane];
+            }
+            if (chunk == prm.stall_chunk &&
+                !warp_wait_flags(lane == 0 ? &g_never_set_word : nullptr, prm.wait_ns)) {
+                lam = __int_as_float(0x7fc00000);  // ran out of time: poison what follows
+                eta = lam;
+                if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
+            } else if (chunk == 0) {
+                lam = cvalid ? prm.lam0[bb * prm.HN + ch] : 1.f;
+                eta = cvalid ? prm.eta0[bb * prm.HN + ch] : 0.f;
+            } else if (chunk == first) {
+                const int64_t slot = tile * (prm.parts - 1) + (part - 1);
+                if (warp_wait_flags(lane == 0 ? prm.part_flags + slot : nullptr, prm.wait_ns)) {
+                    lam = __ldcg(prm.part_state + slot * 64 + lane);
+                    eta = __ldcg(prm.part_state + slot * 64 + 32 + lane);
+                } else {
+                    lam = __int_as_float(0x7fc00000);
+                    eta = lam;
+                    if (lane == 0) atomicOr(&g_error_word, DEV_ERR_TIMEOUT);
+                }
+            }
+            float lo = lam, eo = eta;
+            agg_apply(g, lo, eo);
+            const int ms = (int)(j % W);
+            slots[ms * 64 + lane] = lo;
+            slots[ms * 64 + 32 + lane] = eo;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&carry_bar[ms]);
+            if (chunk == last && part + 1 < prm.parts) {
+                const int64_t slot = tile * (prm.parts - 1) + part;
+                prm.part_state[slot * 64 + lane] = lo;
+                prm.part_state[slot * 64 + 32 + lane] = eo;
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(prm.part_flags + slot, 1u);
+            }
+        };
+
+        // Output group q of this chunk (tokens q*G .. q*G+G-1): claim a free
+        // half of the warp's double buffer (the store that last read it must
+        // be done), fill it, and send it out with TMA bulk-tensor stores.
+        auto group_begin = [&]() -> float * {
+            float *buf = outbuf0 + (group_seq & 1) * (Cfg::OUTBUF_BYTES / 4);
+            if (group_seq >= 2) {
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+            }
+            return buf;
+        };
+        auto group_end = [&](float *buf, int q) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int ty = (int)(t0 + q * G);
+                const int x = (int)(ct * 32);
+                tma_store_3d(&maps.out[0], buf, x, ty, (int)bb);
+                tma_store_3d(&maps.out[1], buf + G * 32, x, ty, (int)bb);
+                if (prm.write_mu) tma_store_3d(&maps.out[2], buf + 2 * G * 32, x, ty, (int)bb);
+                if (prm.write_var) tma_store_3d(&maps.out[3], buf + 3 * G * 32, x, ty, (int)bb);
+                bulk_commit_group();
+            }
+            ++group_seq;
+        };
+        auto put = [&](float *buf, int u, const TokenOut &o) {
+            buf[u * 32 + lane] = o.lam;
+            buf[G * 32 + u * 32 + lane] = o.eta;
+            buf[2 * G * 32 + u * 32 + lane] = o.mu;
+            buf[3 * G * 32 + u * 32 + lane] = o.var;
+        };
+
+        if (t_valid == L) {
+            // Full chunk: read it from shared memory once into registers,
+            // release the stage to the producer right away, then run both
+            // passes from registers.
+            float xa[L], xp[L], xf[L], xb[L];
+#pragma unroll
+            for (int t = 0; t < L; ++t) {
+                const int i = t * 32 + lane;
+                xa[t] = to_f32(stage[i]);
+                xp[t] = to_f32(stage[LC + i]);
+                xf[t] = to_f32(stage[2 * LC + i]);
+                xb[t] = to_f32(stage[3 * LC + i]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            // (1) the chunk's aggregate (renormalised every second token)
+            Agg g = agg_identity();
+#pragma unroll
+            for (int t = 0; t < L; ++t) {
+                agg_push_token(g, xa[t], xp[t], xf[t], xb[t]);
+                if (renorm_after(t)) agg_renorm(g);
+            }
+            agg_renorm(g);
+            // (2) carry
+            float lam, eta;
+            chunk_carry(g, lam, eta);
+            // (3) per-token recursion from the entering state
+#pragma unroll
+            for (int q = 0; q < L / G; ++q) {
+                float *buf = group_begin();
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    const int t = q * G + u;
+                    put(buf, u, filter_token(lam, eta, xa[t], xp[t], xf[t], xb[t]));
+                }
+                group_end(buf, q);
+            }
+        } else {
+            // Ragged last chunk: straight from shared memory, released at the
+            // end; rows past T are clipped by the TMA stores.
+            Agg g = agg_identity();
+#pragma unroll 2
+            for (int t = 0; t < t_valid; ++t) {
+                const int i = t * 32 + lane;
+                agg_push_token(g, to_f32(stage[i]), to_f32(stage[LC + i]), to_f32(stage[2 * LC + i]),
+                               to_f32(stage[3 * LC + i]));
+                if (renorm_after(t)) agg_renorm(g);
+            }
+            agg_renorm(g);
+            float lam, eta;
+            chunk_carry(g, lam, eta);
+            const int ngroups = (t_valid + G - 1) / G;
+#pragma unroll 1
+            for (int q = 0; q < ngroups; ++q) {
+                float *buf = group_begin();
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    const int t = q * G + u;
+                    if (t < t_valid) {
+                        const int i = t * 32 + lane;
+                        put(buf, u, filter_token(lam, eta, to_f32(stage[i]), to_f32(stage[LC + i]),
+                                                 to_f32(stage[2 * LC + i]), to_f32(stage[3 * LC + i])));
+                    }
+                }
+                group_end(buf, q);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+    }
+    // every bulk store of this warp must be complete before the CTA exits
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+}
+
+// The same scan with VEC channels per lane (used with VEC = 2 for bf16
+// inputs: 64-channel tiles, two independent recursion chains per lane).  The
+// one-channel kernel above is kept separate: compiled from this template with
+// VEC = 1 it measured 5% slower on the long fp32 workload.
+template <typename Tin, int L, int W, int NS, int G, int VEC>
+__global__ void __launch_bounds__(32 * (W + 1), 1)
+kla_forward_stream_vec_kernel(const StreamParams prm, const __grid_constant__ FwdMaps maps) {
     using Cfg = StreamTile<Tin, L, W, NS, G, VEC>;
     constexpr int CW = Cfg::CW;
     constexpr int LC = L * CW;
