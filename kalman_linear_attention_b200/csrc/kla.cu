@@ -534,6 +534,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
         if (ok) {
             kla::StreamParams sp;
             sp.lam0 = lambda0; sp.eta0 = eta0;
+            sp.out[0] = lambda_out; sp.out[1] = eta_out; sp.out[2] = mu_out; sp.out[3] = var_out;
             sp.write_mu = mu_out != nullptr; sp.write_var = var_out != nullptr;
             sp.T = T; sp.HN = HN; sp.ntiles = sg.ntiles;
             sp.nct = (int)sg.nct;
