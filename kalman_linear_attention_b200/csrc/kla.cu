@@ -110,23 +110,13 @@ template <typename Tin> constexpr int stream_group() {
 #ifndef KLA_STREAM2_G
 #define KLA_STREAM2_G 8
 #endif
-#ifndef KLA_STREAM2_W_F32
-#define KLA_STREAM2_W_F32 6
-#endif
-#ifndef KLA_STREAM2_G_F32
-#define KLA_STREAM2_G_F32 4
-#endif
-template <typename Tin> constexpr int stream2_warps() { return sizeof(Tin) == 4 ? KLA_STREAM2_W_F32 : KLA_STREAM2_W; }
-template <typename Tin> constexpr int stream2_group() { return sizeof(Tin) == 4 ? KLA_STREAM2_G_F32 : KLA_STREAM2_G; }
+template <typename Tin> constexpr int stream2_warps() { return KLA_STREAM2_W; }
+template <typename Tin> constexpr int stream2_group() { return KLA_STREAM2_G; }
 // 1 disables the two-channel layout (sweeps)
 #ifndef KLA_STREAM2_OFF
 #define KLA_STREAM2_OFF 0
 #endif
-// 1: fp32 inputs take two channels per lane too when the 64-channel tiles
-// still give every SM two rounds of work
-#ifndef KLA_STREAM2_F32
-#define KLA_STREAM2_F32 0
-#endif
+
 
 // Ring stages that fit beside the per-warp output buffers and carry slots.
 template <typename Tin, int VEC = 1>
@@ -381,7 +371,6 @@ struct StreamGeom {
 StreamGeom stream_geom(int64_t B, int64_t T, int64_t HN, size_t esz) {
     StreamGeom g;
     g.vec = (esz == 2 && HN >= 64 && !KLA_STREAM2_OFF) ? 2 : 1;
-    if (KLA_STREAM2_F32 && esz == 4 && HN >= 64 && B * ((HN + 63) / 64) >= 2 * (int64_t)sm_count()) g.vec = 2;
     g.cw = 32 * g.vec;
     g.L = g.vec == 2 ? KLA_STREAM2_L : kSL;
     g.nct = (HN + g.cw - 1) / g.cw;
@@ -556,8 +545,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
             }
             cudaError_t es;
             if (in_dtype == KLA_F32)
-                es = (KLA_STREAM2_F32 && sg.vec == 2) ? launch_forward_stream<float, KLA_STREAM2_F32 ? 2 : 1>(sp, smaps, st)
-                                                      : launch_forward_stream<float>(sp, smaps, st);
+                es = launch_forward_stream<float>(sp, smaps, st);
             else
                 es = sg.vec == 2 ? launch_forward_stream<__nv_bfloat16, 2>(sp, smaps, st)
                                  : launch_forward_stream<__nv_bfloat16>(sp, smaps, st);
@@ -589,11 +577,6 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
                 : launch_forward<__nv_bfloat16, false>(prm, maps, lay.tiles, st);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
-
-// 1: decode steps with eight channels per thread where C % 8 == 0 (sweeps)
-#ifndef KLA_STEP_VEC8
-#define KLA_STEP_VEC8 0
-#endif
 
 KLA_API kla_status_t kla_scan_step(const void *a, const void *p, const void *phi, const void *b,
                                    kla_dtype_t in_dtype, float *lambda_state, float *eta_state,
@@ -628,9 +611,8 @@ KLA_API kla_status_t kla_scan_step(const void *a, const void *p, const void *phi
     for (int k = 0; k < 4; ++k)
         if (outs_p[k] && !aligned16(outs_p[k])) vec = false;
 
-    const bool vec8 = KLA_STEP_VEC8 && vec && (C % 8) == 0;
     const int threads = 256;
-    const int64_t work = vec8 ? C / 8 : (vec ? C / 4 : C);
+    const int64_t work = vec ? C / 4 : C;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((work + threads - 1) / threads, 148 * 16));
     // Programmatic dependent launch: consecutive decode steps overlap the next
     // step's launch and input prefetch with the current step's tail (the
@@ -647,13 +629,11 @@ KLA_API kla_status_t kla_scan_step(const void *a, const void *p, const void *phi
     cfg.numAttrs = 1;
     cudaError_t e;
     if (in_dtype == KLA_F32)
-        e = vec8 ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec8_kernel<float>, prm)
-                 : vec ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec4_kernel<float>, prm)
-                       : cudaLaunchKernelEx(&cfg, kla::kla_step_scalar_kernel<float>, prm);
+        e = vec ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec4_kernel<float>, prm)
+                : cudaLaunchKernelEx(&cfg, kla::kla_step_scalar_kernel<float>, prm);
     else
-        e = vec8 ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec8_kernel<__nv_bfloat16>, prm)
-                 : vec ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec4_kernel<__nv_bfloat16>, prm)
-                       : cudaLaunchKernelEx(&cfg, kla::kla_step_scalar_kernel<__nv_bfloat16>, prm);
+        e = vec ? cudaLaunchKernelEx(&cfg, kla::kla_step_vec4_kernel<__nv_bfloat16>, prm)
+                : cudaLaunchKernelEx(&cfg, kla::kla_step_scalar_kernel<__nv_bfloat16>, prm);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 

@@ -86,48 +86,6 @@ __global__ void __launch_bounds__(256) kla_step_vec4_kernel(const StepParams prm
     }
 }
 
-// Eight channels per thread (two 16-byte loads of each input): C a multiple
-// of 8, the same alignment as the four-channel kernel.
-template <typename Tin>
-__global__ void __launch_bounds__(256) kla_step_vec8_kernel(const StepParams prm) {
-    const int64_t n8 = prm.C >> 3;
-    constexpr int VEC_BYTES = 4 * (int)sizeof(Tin);
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
-         i += (int64_t)gridDim.x * blockDim.x)
-        if ((threadIdx.x & 3) == 0)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                prefetch_l2(static_cast<const char *>(prm.in[k]) + 2 * i * VEC_BYTES);
-    grid_dependency_wait();
-    allow_dependent_launch();
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float4 a[2], p[2], phi[2], b[2], lam[2], eta[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            a[h] = Vec4In<Tin>::load(prm.in[0], 2 * i + h);
-            p[h] = Vec4In<Tin>::load(prm.in[1], 2 * i + h);
-            phi[h] = Vec4In<Tin>::load(prm.in[2], 2 * i + h);
-            b[h] = Vec4In<Tin>::load(prm.in[3], 2 * i + h);
-            lam[h] = reinterpret_cast<const float4 *>(prm.lam)[2 * i + h];
-            eta[h] = reinterpret_cast<const float4 *>(prm.eta)[2 * i + h];
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const TokenOut o0 = filter_token(lam[h].x, eta[h].x, a[h].x, p[h].x, phi[h].x, b[h].x);
-            const TokenOut o1 = filter_token(lam[h].y, eta[h].y, a[h].y, p[h].y, phi[h].y, b[h].y);
-            const TokenOut o2 = filter_token(lam[h].z, eta[h].z, a[h].z, p[h].z, phi[h].z, b[h].z);
-            const TokenOut o3 = filter_token(lam[h].w, eta[h].w, a[h].w, p[h].w, phi[h].w, b[h].w);
-            reinterpret_cast<float4 *>(prm.lam)[2 * i + h] = lam[h];
-            reinterpret_cast<float4 *>(prm.eta)[2 * i + h] = eta[h];
-            if (prm.mu != nullptr)
-                __stcs(reinterpret_cast<float4 *>(prm.mu) + 2 * i + h, make_float4(o0.mu, o1.mu, o2.mu, o3.mu));
-            if (prm.var != nullptr)
-                __stcs(reinterpret_cast<float4 *>(prm.var) + 2 * i + h, make_float4(o0.var, o1.var, o2.var, o3.var));
-        }
-    }
-}
-
 // Any size and alignment: one channel per thread.
 template <typename Tin>
 __global__ void __launch_bounds__(256) kla_step_scalar_kernel(const StepParams prm) {
