@@ -294,7 +294,8 @@ def time_config(kla, w: wl.Workload, device, steps: int, warmup: int, peak: floa
              "value": tc / (ms * 1e-3), "unit": UNIT, "gb_per_s": gbs,
              "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                           "frac_of_nominal": gbs / NOMINAL_HBM_GBS,
-                          "algorithmic_bytes_per_launch": bpt * tc, "bytes_per_token_channel": bpt},
+                          "algorithmic_bytes_per_launch": bpt * tc, "bytes_per_token_channel": bpt,
+                          "traffic": recorded_traffic(w.name, plan[0])},
              "kernel": FORWARD_KERNELS[plan[0]], "launches_per_call": plan[1],
              "timing": "median of per-launch CUDA events, L2 flushed (256 MB write) between launches"}
     return entry, x
@@ -374,7 +375,8 @@ def time_lti(kla, device, steps: int, warmup: int, peak: float, tokens: int = 0)
             "kernel": {1: "kla_lti_seq_kernel (one thread per channel)",
                        2: "kla_lti_stream_kernel (channel-owning streaming, blocked convolutions)"}[plan[0]],
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "algorithmic_bytes_per_launch": bpt * tc, "bytes_per_token_channel": bpt},
+                         "algorithmic_bytes_per_launch": bpt * tc, "bytes_per_token_channel": bpt,
+                         "traffic": recorded_traffic("lti" if not tokens else f"lti@T={tokens}", plan[0])},
             "max_rel_err_lambda_vs_oracle": err_lti,
             "general_scan_same_problem": {
                 "ms": gms, "value": tc / (gms * 1e-3), "bytes_per_token_channel": 32,
@@ -414,7 +416,9 @@ def time_attention(kla, device, steps: int, warmup: int, peak: float, W: int = 6
             "kernel": "kla_attention_kernel", "weights_per_s": write_bytes / 4 / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "algorithmic_bytes_per_launch": write_bytes + read_bytes,
-                         "bytes": f"{W}*{W}*4 written per channel and window + a, p (bf16) and lambda read"},
+                         "bytes": f"{W}*{W}*4 written per channel and window + a, p (bf16) and lambda read",
+                         "traffic": recorded_traffic("attention" if not rows and W == 64 else
+                                                     f"attention@B={w.B},W={W}", 1)},
             "timing": "median of per-launch CUDA events (8.6 GB written per launch, larger than L2)"}
 
 

@@ -100,7 +100,9 @@ template <typename Tin> constexpr int stream_group() {
 // KLA_STREAM2_L-token chunks (the same registers per thread as 32 tokens x
 // one channel), chunk warps and output group.  On the LM-layer shape: 5%
 // faster than one channel per lane with 8-token output groups, no faster
-// with 4, slower with 6 chunk warps.
+// with 4, slower with 6 chunk warps; one 16-token group per chunk in a
+// single buffer (KLA_STREAM2_NBUF, half the bulk stores) 2% faster than two
+// double-buffered 8-token groups.
 #ifndef KLA_STREAM2_L
 #define KLA_STREAM2_L 16
 #endif
@@ -108,7 +110,7 @@ template <typename Tin> constexpr int stream_group() {
 #define KLA_STREAM2_W 7
 #endif
 #ifndef KLA_STREAM2_G
-#define KLA_STREAM2_G 8
+#define KLA_STREAM2_G 16
 #endif
 template <typename Tin> constexpr int stream2_warps() { return KLA_STREAM2_W; }
 template <typename Tin> constexpr int stream2_group() { return KLA_STREAM2_G; }
@@ -126,7 +128,8 @@ constexpr int stream_stages() {
     constexpr int L = VEC == 1 ? kSL : KLA_STREAM2_L;
     constexpr int CW = 32 * VEC;
     const int stage = 4 * L * CW * (int)sizeof(Tin);
-    const int fixed = W * 2 * 4 * G * CW * 4 + W * 2 * CW * 4 + W * 8 + 2048;
+    constexpr int NBUF = VEC == 1 ? KLA_STREAM_NBUF : KLA_STREAM2_NBUF;
+    const int fixed = W * NBUF * 4 * G * CW * 4 + W * 2 * CW * 4 + W * 8 + 2048;
     const int ns = (KLA_STREAM_SMEM - fixed) / stage;
     return ns > KLA_STREAM_MAX_STAGES ? KLA_STREAM_MAX_STAGES : ns;
 }
@@ -255,6 +258,28 @@ cudaError_t ensure_smem_attr(K kernel, int smem) {
     return e;
 }
 
+// Launch of a scan kernel that follows a workspace clear on the stream.  With
+// `after_clear` it is the clear kernel's programmatic dependent: it becomes
+// resident while the clear runs, and its griddepcontrol.wait (which every
+// kernel launched this way executes before it touches the workspace) holds it
+// until the clear is done.  Everything before the clear on the stream has
+// completed by the time the clear starts, so the scan's inputs are ready.
+template <typename... P, typename... A>
+cudaError_t launch_scan_kernel(void (*kernel)(P...), int64_t grid, int threads, size_t smem,
+                               cudaStream_t stream, bool after_clear, A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_clear ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 template <typename Tin, bool TMA>
 cudaError_t launch_forward(const FwdParams &prm, const FwdMaps &maps, int64_t tiles,
                            cudaStream_t stream) {
@@ -262,8 +287,7 @@ cudaError_t launch_forward(const FwdParams &prm, const FwdMaps &maps, int64_t ti
     auto kernel = kla::kla_forward_kernel<Tin, kL, kCW, kR, TMA>;
     cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    kernel<<<(unsigned)tiles, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
-    return cudaGetLastError();
+    return launch_scan_kernel(kernel, tiles, Cfg::THREADS, Cfg::SMEM, stream, true, prm, maps);
 }
 
 int sm_count() {
@@ -298,7 +322,7 @@ cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &m
         auto kernel = kla::kla_forward_stream_vec_kernel<Tin, L, W, NS, G, VEC>;
         cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
         if (e != cudaSuccess) return e;
-        kernel<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM, stream>>>(prm, maps);
+        return launch_scan_kernel(kernel, grid, Cfg::THREADS, Cfg::SMEM, stream, prm.parts > 1, prm, maps);
     }
     return cudaGetLastError();
 }

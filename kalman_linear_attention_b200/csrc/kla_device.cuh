@@ -166,6 +166,22 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch
+// ---------------------------------------------------------------------------
+// A kernel launched with programmatic stream serialization may become
+// resident as soon as every CTA of the kernel before it on the stream has
+// executed `griddepcontrol.launch_dependents` (or exited); `griddepcontrol.wait`
+// then blocks the calling thread until that kernel has completed and its
+// writes are visible.  In a kernel launched without the attribute the wait
+// returns at once.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Time and flags
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t globaltimer_ns() {

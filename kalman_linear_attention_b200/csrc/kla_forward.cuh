@@ -126,6 +126,7 @@ kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
     const int r = tid / CW;
 
     // ---- 1. ticket and load ------------------------------------------------
+    grid_dependency_wait();  // the workspace clear before this kernel is done
     if (tid == 0) {
         const unsigned ticket = atomicAdd(prm.ticket, 1u);
         *s_ticket = ticket;
@@ -322,7 +323,11 @@ kla_forward_kernel(const FwdParams prm, const __grid_constant__ FwdMaps maps) {
 }
 
 // Zero the ticket counter and the ready flags of a workspace.
+// Zeroes a workspace's counters and flags.  The scan kernel that follows it
+// may be launched as its programmatic dependent: it becomes resident and sets
+// up while this kernel runs, and waits for it before touching the workspace.
 __global__ void kla_clear_kernel(uint4 *p, int64_t n16) {
+    allow_dependent_launch();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16;
          i += (int64_t)gridDim.x * blockDim.x)
         p[i] = make_uint4(0u, 0u, 0u, 0u);

@@ -29,7 +29,9 @@
 // A lane owns VEC consecutive channels (CW = 32 VEC per tile): with VEC = 2
 // (bf16 inputs: 64-channel tiles, 16-token chunks, the same registers per
 // thread) every lane runs two independent recursion chains side by side, and
-// one 32-bit shared load brings a token's two bf16 values of an input.
+// one 32-bit shared load brings a token's two bf16 values of an input; its
+// output box is the whole chunk (G = L), single-buffered: the next chunk's
+// first pass runs while the bulk stores read it out.
 //
 // Within a tile no global flags, fences or look-back: the W warps overlap
 // their passes while the producer keeps HBM busy.  Chunk aggregates are formed
@@ -98,6 +100,15 @@ struct StreamChunk {
     int first, last;               // chunks of the run
 };
 
+// Output buffers per chunk warp: 2 (double-buffered output groups) or 1 (a
+// group waits for the bulk stores of the previous one to have read it).
+#ifndef KLA_STREAM_NBUF
+#define KLA_STREAM_NBUF 2
+#endif
+#ifndef KLA_STREAM2_NBUF
+#define KLA_STREAM2_NBUF 1
+#endif
+
 template <typename Tin, int L, int W, int NS, int G, int VEC = 1>
 struct StreamTile {
     // Chunk j sits in stage j % NS and is handled by warp j % W.  With
@@ -113,8 +124,10 @@ struct StreamTile {
     static constexpr int STAGE_BYTES = 4 * L * CW * (int)sizeof(Tin);
     static constexpr int OUTBOX_BYTES = G * CW * 4;                 // one output, one group
     static constexpr int OUTBUF_BYTES = 4 * OUTBOX_BYTES;           // four outputs
-    static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][2][4][G][CW] fp32
-    static constexpr int CARRY_OFF = OUT_OFF + W * 2 * OUTBUF_BYTES; // [W][2][CW] fp32
+    static constexpr int NBUF = VEC == 1 ? KLA_STREAM_NBUF : KLA_STREAM2_NBUF;
+    static_assert(NBUF == 1 || NBUF == 2, "one or two output buffers per warp");
+    static constexpr int OUT_OFF = NS * STAGE_BYTES;                 // [W][NBUF][4][G][CW] fp32
+    static constexpr int CARRY_OFF = OUT_OFF + W * NBUF * OUTBUF_BYTES; // [W][2][CW] fp32
     static constexpr int META_OFF = CARRY_OFF + W * 2 * CW * 4;      // per stage: unit (int64), chunk (int64)
     static constexpr int BAR_OFF = align_up(META_OFF + NS * 16, 128); // full, empty, carry
     static constexpr int SMEM = align_up(BAR_OFF + (2 * NS + W) * 8, 128);
@@ -238,7 +251,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 
     // ------------------------------------------------------------ chunk warps
     const int w = warp - 1;
-    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
+    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * Cfg::NBUF * Cfg::OUTBUF_BYTES);
     int group_seq = 0;  // output groups this warp has committed (bulk groups are per thread: lane 0)
 #pragma unroll 1
     for (int64_t j = w;; j += W) {
@@ -311,9 +324,9 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
         // half of the warp's double buffer (the store that last read it must
         // be done), fill it, and send it out with TMA bulk-tensor stores.
         auto group_begin = [&]() -> float * {
-            float *buf = outbuf0 + (group_seq & 1) * (Cfg::OUTBUF_BYTES / 4);
-            if (group_seq >= 2) {
-                if (lane == 0) bulk_wait_group_read<1>();
+            float *buf = outbuf0 + (group_seq & (Cfg::NBUF - 1)) * (Cfg::OUTBUF_BYTES / 4);
+            if (group_seq >= Cfg::NBUF) {
+                if (lane == 0) bulk_wait_group_read<Cfg::NBUF - 1>();
                 __syncwarp();
             }
             return buf;
@@ -445,6 +458,7 @@ kla_forward_stream_vec_kernel(const StreamParams prm, const __grid_constant__ Fw
         fence_mbar_init();
     }
     __syncthreads();
+    grid_dependency_wait();  // a workspace clear launched before this kernel is done
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -504,7 +518,7 @@ kla_forward_stream_vec_kernel(const StreamParams prm, const __grid_constant__ Fw
 
     // ------------------------------------------------------------ chunk warps
     const int w = warp - 1;
-    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * 2 * Cfg::OUTBUF_BYTES);
+    float *outbuf0 = reinterpret_cast<float *>(smem + Cfg::OUT_OFF + w * Cfg::NBUF * Cfg::OUTBUF_BYTES);
     int group_seq = 0;  // output groups this warp has committed (bulk groups are per thread: lane 0)
     const int lc = lane * VEC;  // this lane's first channel within a tile
 #pragma unroll 1
@@ -601,9 +615,9 @@ kla_forward_stream_vec_kernel(const StreamParams prm, const __grid_constant__ Fw
         // half of the warp's double buffer (the store that last read it must
         // be done), fill it, and send it out with TMA bulk-tensor stores.
         auto group_begin = [&]() -> float * {
-            float *buf = outbuf0 + (group_seq & 1) * (Cfg::OUTBUF_BYTES / 4);
-            if (group_seq >= 2) {
-                if (lane == 0) bulk_wait_group_read<1>();
+            float *buf = outbuf0 + (group_seq & (Cfg::NBUF - 1)) * (Cfg::OUTBUF_BYTES / 4);
+            if (group_seq >= Cfg::NBUF) {
+                if (lane == 0) bulk_wait_group_read<Cfg::NBUF - 1>();
                 __syncwarp();
             }
             return buf;

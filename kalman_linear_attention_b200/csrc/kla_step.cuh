@@ -44,12 +44,6 @@ template <> struct Vec4In<__nv_bfloat16> {
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" :: "l"(p));
 }
-__device__ __forceinline__ void grid_dependency_wait() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void allow_dependent_launch() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 // Four channels per thread; every pointer 16-byte aligned (8 for bf16
 // inputs) and C a multiple of 4.
