@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -76,11 +77,20 @@ def max_over_ranks(x: float, dist_mod=None) -> float:
     return float(t.item())
 
 
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources with comments and blank space removed, so
+    that recorded profiler figures stay attached to the code they measured
+    and survive edits of the comments only."""
     h = hashlib.sha256()
     for f in sorted(os.listdir(CSRC)):
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        if not f.endswith((".cu", ".cuh", ".h")):
+            continue
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            code = " ".join(_COMMENT.sub(" ", fh.read()).split())
+        h.update(f.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 

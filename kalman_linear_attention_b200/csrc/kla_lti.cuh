@@ -33,9 +33,10 @@
 // the whole sequence; a producer warp streams chunks into a ring of shared-
 // memory stages with TMA; chunk warps take chunks round-robin, compute (1)
 // and (2) without waiting, take the entering state from the previous chunk's
-// warp (mbarrier), hand on the exit, and run (4) into double-buffered output
-// boxes stored with TMA.  Rows past T arrive as zeros (TMA fill) and are
-// clipped on store, so a ragged last chunk needs no separate path.  Tiles
+// warp (mbarrier), hand on the exit, and run (4) straight from registers to
+// global memory: one coalesced 128-byte streaming store per output and token
+// (measured faster here than output boxes stored with TMA).  Rows past T
+// arrive as zeros (TMA fill) and are not stored.  Tiles
 // that do not spread evenly over the SMs are cut into runs taken by ticket,
 // as in the general streaming scan; run boundaries hand on fp64 states.  The
 // producer passes each chunk's tile coordinates in the stage's metadata.

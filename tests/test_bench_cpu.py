@@ -47,3 +47,28 @@ def test_defaults_and_byte_counts():
     assert bench.algorithmic_bytes_per_tc(bench.wl.WORKLOADS["lm_layer"]) == 24
     assert bench.backward_bytes_per_tc(bench.wl.WORKLOADS["lm_layer"]) == 36
     assert bench.decode_bytes_per_channel(bench.wl.WORKLOADS["decode"]) == 40
+
+
+def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    """Recorded DRAM traffic stays attached to the code it measured: editing
+    a comment keeps the hash, editing code changes it."""
+    src = "// a kernel\n__global__ void k(float *x) { x[0] = 1.f; /* one store */ }\n"
+    (tmp_path / "k.cuh").write_text(src)
+    monkeypatch.setattr(bench, "CSRC", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    (tmp_path / "k.cuh").write_text(src.replace("a kernel", "the kernel").replace("one store", "1 store"))
+    assert bench.kernel_source_hash() == h0
+    (tmp_path / "k.cuh").write_text(src.replace("1.f", "2.f"))
+    assert bench.kernel_source_hash() != h0
+
+
+def test_recorded_traffic_entries_are_complete():
+    """Every entry of the committed traffic record names its kernel, the
+    source hash it was taken on, and read + write bytes that add up."""
+    with open(bench.TRAFFIC_FILE) as f:
+        d = json.load(f)
+    assert {"long", "long:backward", "lm_layer", "stiff", "lti", "attention"} <= set(d)
+    for e in d.values():
+        assert e["kernel"] in (1, 2) and len(e["kernel_sha"]) == 16
+        rw = e["dram_read_bytes_per_launch"] + e["dram_write_bytes_per_launch"]
+        assert abs(rw - e["dram_bytes_per_launch"]) < 1.0
