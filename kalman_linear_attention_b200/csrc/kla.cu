@@ -322,7 +322,7 @@ cudaError_t launch_forward_stream(const kla::StreamParams &prm, const FwdMaps &m
         auto kernel = kla::kla_forward_stream_vec_kernel<Tin, L, W, NS, G, VEC>;
         cudaError_t e = ensure_smem_attr(kernel, Cfg::SMEM);
         if (e != cudaSuccess) return e;
-        return launch_scan_kernel(kernel, grid, Cfg::THREADS, Cfg::SMEM, stream, prm.parts > 1, prm, maps);
+        return launch_scan_kernel(kernel, grid, Cfg::THREADS, Cfg::SMEM, stream, prm.ticket != nullptr, prm, maps);
     }
     return cudaGetLastError();
 }
@@ -391,6 +391,7 @@ struct StreamGeom {
     int vec, cw, L;
     int64_t ntiles, nct, nchunks;
     int parts;
+    bool ticketed;  // units taken by ticket (a workspace counter) rather than round-robin
 };
 StreamGeom stream_geom(int64_t B, int64_t T, int64_t HN, size_t esz) {
     StreamGeom g;
@@ -401,6 +402,13 @@ StreamGeom stream_geom(int64_t B, int64_t T, int64_t HN, size_t esz) {
     g.ntiles = B * g.nct;
     g.nchunks = (T + g.L - 1) / g.L;
     g.parts = stream_parts(g.ntiles, g.nchunks, g.vec == 2 ? 1 : 2);
+    // Whole tiles are ticketed too when there are more than the SMs and each
+    // is at least 8 chunks long: a CTA on a faster SM then takes more of them
+    // (CTAs with equal round-robin shares finish up to 30% apart on some
+    // shapes: B=256, H*N=512, T=512 fp32 12% faster ticketed, the LM-layer
+    // shape at B=37 8%); shorter tiles stay round-robin (the stiff shape,
+    // 4 chunks per tile, 2-3% slower ticketed).
+    g.ticketed = g.parts > 1 || (g.ntiles > (int64_t)sm_count() && g.nchunks >= 8);
     return g;
 }
 
@@ -566,6 +574,11 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
                 sp.part_flags = reinterpret_cast<unsigned *>(ws + sw.flags_off);
                 sp.part_state = reinterpret_cast<float *>(ws + sw.state_off);
                 if (launch_clear(ws, sw.clear_bytes, st) != cudaSuccess) return KLA_ERR_CUDA;
+            } else if (sg.ticketed) {
+                if (launch_clear(ws, stream_ws_layout(sp.ntiles, 1, sg.cw).clear_bytes, st) != cudaSuccess)
+                    return KLA_ERR_CUDA;
+            } else {
+                sp.ticket = nullptr;  // round-robin units, no workspace
             }
             cudaError_t es;
             if (in_dtype == KLA_F32)
@@ -701,7 +714,7 @@ KLA_API kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int6
     *kernel = forward_kernel_choice(B, T, HN, dtype_size(in_dtype), a, p, phi, b, nullptr, nullptr, nullptr,
                                     nullptr);
     *launches = 2;  // chunked kernel: workspace clear + scan
-    if (*kernel == 2) *launches = stream_geom(B, T, HN, dtype_size(in_dtype)).parts > 1 ? 2 : 1;
+    if (*kernel == 2) *launches = stream_geom(B, T, HN, dtype_size(in_dtype)).ticketed ? 2 : 1;
     return KLA_OK;
 }
 

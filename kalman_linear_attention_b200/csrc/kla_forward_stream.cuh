@@ -37,8 +37,9 @@
 // their passes while the producer keeps HBM busy.  Chunk aggregates are formed
 // and applied exactly as in kla_forward_kernel (one thread's run = the whole
 // chunk here).  A CTA with more than one work unit processes them one after
-// another.  When tiles do not divide evenly over the SMs, each tile's
-// sequence is cut into a few runs taken by ticket, run-major, so that a run
+// another, taking them by ticket when they are long enough for a faster SM
+// to gain by taking more.  When tiles do not divide evenly over the SMs, each
+// tile's sequence is cut into a few runs taken by ticket, run-major, so that a run
 // after the first finds the state published by the previous run (one bounded
 // global wait per run; deadlock-free because a run only waits on a run with a
 // smaller ticket).  Every wait is bounded by the wait limit (a timeout
@@ -77,14 +78,15 @@ struct StreamParams {
     int nchunks;                   // ceil(T / L)
     int write_mu, write_var;       // outputs 2 / 3 requested
     uint64_t wait_ns;
-    // Work units.  parts == 1: unit = tile, CTA c takes tiles c, c + grid, ...
-    // parts > 1: each tile's chunks are cut into `parts` consecutive runs of
-    // chunks_per_part; unit u = part * ntiles + tile is taken by ticket (part
-    // major), and a run after the first enters with the state the previous run
-    // of the same tile published in part_state (flag part_flags).
+    // Work units.  parts == 1: unit = tile, taken by ticket or (ticket null)
+    // round-robin, CTA c taking tiles c, c + grid, ...  parts > 1: each
+    // tile's chunks are cut into `parts` consecutive runs of chunks_per_part;
+    // unit u = part * ntiles + tile is taken by ticket (part major), and a run
+    // after the first enters with the state the previous run of the same tile
+    // published in part_state (flag part_flags).
     int parts, chunks_per_part;
     int64_t nunits;                // ntiles * parts
-    unsigned *ticket;              // parts > 1: unit counter (zeroed per call)
+    unsigned *ticket;              // unit counter (zeroed per call); null: round-robin units
     unsigned *part_flags;          // [ntiles][parts - 1], zeroed per call
     float *part_state;             // [ntiles][parts - 1][2][CW]
     int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
@@ -228,7 +230,7 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 #pragma unroll 1
             for (int c = first; c <= last; ++c) load(u, c, bb, ct);
         };
-        if (prm.parts == 1) {
+        if (prm.ticket == nullptr) {
 #pragma unroll 1
             for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
         } else {
@@ -495,7 +497,7 @@ kla_forward_stream_vec_kernel(const StreamParams prm, const __grid_constant__ Fw
 #pragma unroll 1
             for (int c = first; c <= last; ++c) load(u, c, bb, ct);
         };
-        if (prm.parts == 1) {
+        if (prm.ticket == nullptr) {
 #pragma unroll 1
             for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
         } else {

@@ -270,6 +270,35 @@ def test_special_cases_decode(kind):
     assert np.max(np.abs(lam.double().cpu().numpy() - ref["lam"][:, -1]) / ref["lam"][:, -1]) <= 1e-5
 
 
+@pytest.mark.parametrize("family,shape", [
+    ("stiff", dict(B=160, T=300, H=1, N=32)),        # 160 tiles of 32 channels, 10 chunks, ragged
+    ("lm_layer", dict(B=5, T=200, H=16, N=128)),     # bf16: 160 tiles of 64 channels, 13 chunks
+])
+def test_ticketed_whole_tiles_parity(family, shape):
+    """More tiles than SMs, one run each, long enough to be taken by ticket
+    (a CTA on a faster SM takes more of them): the plan reports the clear
+    launch, every element matches the oracle, and a second call is
+    bit-identical whatever order the tickets were taken in."""
+    kla = _kla()
+    w = wl.WORKLOADS[family].with_shape(**shape)
+    x = wl.generate(w)
+    dt = parity.torch_dtype(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV).to(dt) for k in wl.INPUT_NAMES}
+    for k in ("lam0", "eta0"):
+        d[k] = torch.from_numpy(x[k]).to(DEV)
+    assert kla.forward_plan(d["a"], d["p"], d["phi"], d["b"]) == (2, 2)
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out)}
+    xin = {k: torch.from_numpy(x[k]).to(dt).double().numpy() for k in wl.INPUT_NAMES}
+    ref = oracle.forward(xin["a"], xin["p"], xin["phi"], xin["b"], x["lam0"], x["eta0"], threads=8)
+    parity.assert_parity(got, ref, parity.RTOL[w.dtype], time_axis=1, what=f"{family} ticketed tiles")
+    again = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    for a_, b_ in zip(out, again):
+        assert torch.equal(a_, b_)
+
+
 def test_run_split_parity():
     """320 tiles of 32 channels do not divide evenly over the SMs, so the
     streaming kernel cuts each tile's sequence into runs taken by ticket; a

@@ -9,8 +9,8 @@ previous one left there: the streaming kernel with its tiles split into runs
 (ticket, run flags and run-boundary states), the chunked kernel forced on a
 shape the streaming kernel would take (ticket, per-chunk flags, aggregates and
 carried states: the whole layout), the chunked kernel chosen by geometry, the
-streaming kernel without a split, and the split again after the chunked
-kernel's layout.  Every call is checked against the oracle and, bit for bit,
+streaming kernel without a split (whole tiles by ticket, then round-robin),
+and the split again after the chunked kernel's layout.  Every call is checked against the oracle and, bit for bit,
 against kla_scan_forward with its own workspace.  Collected last on purpose."""
 import pytest
 import torch
@@ -30,8 +30,10 @@ CASES = [
     (wl.WORKLOADS["lm_layer"].with_shape(B=2, T=1500, H=4, seed=22), 1),
     # H*N = 24 < 32: the chunked kernel by geometry
     (wl.WORKLOADS["tiny"].with_shape(B=3, H=3, N=8, T=333, seed=23), 0),
-    # the streaming kernel without a run split
+    # the streaming kernel with whole tiles taken by ticket (256 tiles of 22 chunks)
     (wl.WORKLOADS["stiff"].with_shape(B=16, T=700, seed=24), 0),
+    # the streaming kernel with whole tiles round-robin (7 chunks per tile): no workspace
+    (wl.WORKLOADS["stiff"].with_shape(B=16, T=200, seed=27), 0),
     # the chunked kernel on the first shape, then the run split again on
     # what the chunked kernel left behind
     (wl.WORKLOADS["tiny"].with_shape(B=10, H=8, N=128, T=700, seed=25), 1),
@@ -66,7 +68,7 @@ def test_static_scratch_reused_across_calls_and_kernels():
     for w, force in CASES:
         x, pri, plan, outs, ref = _run(kla, w, force)
         kernel = plan[0]
-        # the streaming kernel launches twice (clear + scan) when it splits tiles into runs
+        # the streaming kernel launches twice (clear + scan) when it takes its units by ticket
         seen.add(("stream" if kernel == 2 else "chunked", plan[1]))
         got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, outs)}
         exp = oracle.forward(x["a"], x["p"], x["phi"], x["b"], pri["lam0"], pri["eta0"], threads=8)
