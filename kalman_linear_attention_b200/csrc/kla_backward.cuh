@@ -47,7 +47,8 @@
 //       chunk and hand the earlier one its carry, (3) re-run the exact
 //       recursion from the carry and store the four input gradients through
 //       double-buffered TMA-store boxes.  Tiles that do not balance over the
-//       SMs are cut into runs taken by ticket (the latest run first).
+//       SMs are cut into runs taken by ticket (the latest run first); more
+//       tiles than SMs, each long enough, are taken whole by ticket.
 //   kla_backward_seq_kernel  one thread per channel walking the sequence
 //       backwards with plain loads; for shapes the TMA geometry does not fit.
 #pragma once
@@ -113,7 +114,7 @@ struct BwdParams {
     // with the carry that run r + 1 published in part_state (flag part_flags).
     int parts, chunks_per_part;
     int64_t nunits;
-    unsigned *ticket;
+    unsigned *ticket;              // unit counter (zeroed per call); null: round-robin units
     unsigned *part_flags;          // [ntiles][parts - 1]
     float *part_state;             // [ntiles][parts - 1][2][32]
     int64_t stall_chunk;           // test hook: this chunk's carry waits on a flag nothing sets (-1: off)
@@ -242,7 +243,7 @@ kla_backward_stream_kernel(const BwdParams prm, const __grid_constant__ BwdMaps 
                 load(m);
             }
         };
-        if (prm.parts == 1) {
+        if (prm.ticket == nullptr) {  // round-robin units
 #pragma unroll 1
             for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
         } else {

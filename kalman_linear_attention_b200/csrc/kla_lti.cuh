@@ -38,7 +38,9 @@
 // (measured faster here than output boxes stored with TMA).  Rows past T
 // arrive as zeros (TMA fill) and are not stored.  Tiles
 // that do not spread evenly over the SMs are cut into runs taken by ticket,
-// as in the general streaming scan; run boundaries hand on fp64 states.  The
+// as in the general streaming scan (and, as there, more tiles than SMs, each
+// long enough, are taken whole by ticket); run boundaries hand on fp64
+// states.  The
 // producer passes each chunk's tile coordinates in the stage's metadata.
 #pragma once
 
@@ -58,7 +60,7 @@ struct LtiParams {
     uint64_t wait_ns;
     int parts, chunks_per_part;
     int64_t nunits;
-    unsigned *ticket;
+    unsigned *ticket;              // unit counter (zeroed per call); null: round-robin units
     unsigned *part_flags;          // [ntiles][parts - 1]
     double *part_state;            // [ntiles][parts - 1][2][32]
 };
@@ -169,7 +171,7 @@ kla_lti_stream_kernel(const LtiParams prm, const __grid_constant__ LtiMaps maps)
                 tma_load_3d(stage + LC, &maps.in[1], m.ct * 32, c * L, m.bb, &full[s]);
             }
         };
-        if (prm.parts == 1) {
+        if (prm.ticket == nullptr) {  // round-robin units
 #pragma unroll 1
             for (int64_t u = blockIdx.x; u < prm.nunits; u += gridDim.x) unit_chunks(u);
         } else {

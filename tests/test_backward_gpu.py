@@ -163,6 +163,18 @@ def test_backward_run_split():
     assert_grad_parity(got, ref, parity.RTOL["f32"], what="run split")
 
 
+def test_backward_ticketed_whole_tiles():
+    """More tiles than SMs, one run each, long enough to be taken whole by
+    ticket: the plan reports the clear launch and the gradients match the
+    oracle."""
+    kla = _kla()
+    w = wl.WORKLOADS["stiff"].with_shape(B=160, T=300, H=1, N=32)  # 160 tiles, 19 chunks
+    a = torch.empty((w.B, w.T, w.H, w.N), device=DEV)
+    assert kla.backward_plan(a, a) == (2, 2)
+    got, ref = run_backward(w)
+    assert_grad_parity(got, ref, parity.RTOL["f32"], what="ticketed whole tiles")
+
+
 def test_backward_empty_and_zero_length():
     kla = _kla()
     z = torch.empty((2, 0, 1, 32), device=DEV)

@@ -122,6 +122,17 @@ def test_lti_kernels_and_run_split():
     _check(got1, ref, ref_abs, 1e-5, "one thread per channel")
 
 
+def test_lti_ticketed_whole_tiles():
+    """160 tiles of 32 channels, one run each, taken whole by ticket: the plan
+    reports the clear launch and every element matches the oracle's filter."""
+    import kalman_linear_attention_b200 as kla
+    w, x = _problem(160, 300, 1, 32, "f32", seed=91)
+    d, outs = _gpu(kla, w, x)
+    assert kla.lti_plan(d["phi"], d["b"]) == (2, 2)
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, outs)}
+    _check(got, _filter_p0(x), _abs_terms(x, lti=False), 1e-5, "ticketed whole tiles")
+
+
 def test_lti_agrees_with_general_scan_and_skips_outputs():
     """Same inputs through kla_scan_forward (a broadcast over time, p = 0):
     both agree with the oracle (64 tokens: the general scan repeats the same
