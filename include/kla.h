@@ -135,8 +135,10 @@ kla_status_t kla_scan_forward(const void *a, const void *p, const void *phi, con
  * chunks exchange carries through the workspace, 2 = the channel-owning
  * streaming kernel; *launches = the kernel launches one call enqueues (2 for
  * the chunked kernel, preceded by a workspace clear; 1 or 2 for the
- * streaming kernel, 2 when it splits tiles into runs).  0 and 0 for an empty
- * problem.  Honours kla_debug_force_forward_kernel.
+ * streaming kernel, 2 when it takes its work units by ticket from the
+ * workspace: tiles split into runs, or more tiles than SMs, each at least 8
+ * chunks long).  0 and 0 for an empty problem.  Honours
+ * kla_debug_force_forward_kernel.
  */
 kla_status_t kla_scan_forward_plan(int64_t B, int64_t T, int64_t H, int64_t N, kla_dtype_t in_dtype,
                                    const void *a, const void *p, const void *phi, const void *b,
