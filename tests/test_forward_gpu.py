@@ -299,6 +299,26 @@ def test_ticketed_whole_tiles_parity(family, shape):
         assert torch.equal(a_, b_)
 
 
+def test_run_split_parity_two_channels():
+    """bf16, 320 tiles of 64 channels: the two-channel kernel cuts each tile
+    into 4 runs of decreasing length (the last tickets the shortest); every
+    element against the oracle on the bf16-rounded inputs."""
+    kla = _kla()
+    w = wl.WORKLOADS["lm_layer"].with_shape(B=10, T=1024, H=16, N=128)
+    x = wl.generate(w)
+    d = {k: torch.from_numpy(x[k]).to(DEV).to(torch.bfloat16) for k in wl.INPUT_NAMES}
+    for k in ("lam0", "eta0"):
+        d[k] = torch.from_numpy(x[k]).to(DEV)
+    assert kla.forward_plan(d["a"], d["p"], d["phi"], d["b"]) == (2, 2)
+    out = kla.scan_forward(d["a"], d["p"], d["phi"], d["b"], d["lam0"], d["eta0"])
+    torch.cuda.synchronize()
+    assert kla.get_error() == 0
+    got = {k: o.double().cpu().numpy() for k, o in zip(parity.OUTPUTS, out)}
+    xin = {k: d[k].double().cpu().numpy() for k in wl.INPUT_NAMES}
+    ref = oracle.forward(xin["a"], xin["p"], xin["phi"], xin["b"], x["lam0"], x["eta0"], threads=8)
+    parity.assert_parity(got, ref, parity.RTOL["f32"], time_axis=1, what="two-channel run split")
+
+
 def test_run_split_parity():
     """320 tiles of 32 channels do not divide evenly over the SMs, so the
     streaming kernel cuts each tile's sequence into runs taken by ticket; a
