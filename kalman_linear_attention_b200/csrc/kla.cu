@@ -575,7 +575,7 @@ KLA_API kla_status_t kla_scan_forward(const void *a, const void *p, const void *
             sp.wait_ns = g_wait_ns.load();
             sp.stall_chunk = g_stall_chunk.load() >= 0 ? g_stall_chunk.load() * kL / sg.L : -1;
             sp.parts = sg.parts;
-            sp.chunks_per_part = (sp.nchunks + sp.parts - 1) / sp.parts;  // equal runs (one-channel kernel)
+            sp.chunks_per_part = (sp.nchunks + sp.parts - 1) / sp.parts;  // (the kernels cut runs 4:3:2:1)
             sp.nunits = sp.ntiles * sp.parts;
             sp.ticket = reinterpret_cast<unsigned *>(ws);
             sp.part_flags = nullptr;

@@ -80,10 +80,13 @@ struct StreamParams {
     uint64_t wait_ns;
     // Work units.  parts == 1: unit = tile, taken by ticket or (ticket null)
     // round-robin, CTA c taking tiles c, c + grid, ...  parts > 1: each
-    // tile's chunks are cut into `parts` consecutive runs of chunks_per_part;
-    // unit u = part * ntiles + tile is taken by ticket (part major), and a run
-    // after the first enters with the state the previous run of the same tile
-    // published in part_state (flag part_flags).
+    // tile's chunks are cut into `parts` consecutive runs of decreasing length
+    // (guided_start); unit u = part * ntiles + tile is taken by ticket (part
+    // major), and a run after the first enters with the state the previous
+    // run of the same tile published in part_state (flag part_flags).
+    // chunks_per_part (equal runs) is no longer read by these kernels; the
+    // field stays because this kernel's speed follows its register
+    // allocation, which follows the parameter block's layout.
     int parts, chunks_per_part;
     int64_t nunits;                // ntiles * parts
     unsigned *ticket;              // unit counter (zeroed per call); null: round-robin units
@@ -168,6 +171,16 @@ __device__ __forceinline__ void sts_vec(float *dst, const float (&v)[2]) {
     *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
 }
 
+// Start chunk of run r of P over n chunks, run lengths in the ratio
+// P : P-1 : ... : 1: the tickets taken last are the shortest runs, so the
+// CTAs finish closer together (1-5% faster than equal runs on LM-layer and
+// run-split fp32 shapes).  n >= P (P + 1) / 2 keeps every run non-empty (the
+// host cuts runs only for n >= 8 P).
+__device__ __forceinline__ int guided_start(int r, int P, int n) {
+    const int k = P - r;
+    return n - (int)(((int64_t)n * (k * (k + 1) / 2)) / (P * (P + 1) / 2));
+}
+
 template <typename Tin, int L, int W, int NS, int G>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
 kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMaps maps) {
@@ -225,8 +238,8 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
             const int part = (int)(u / prm.ntiles);
             const int bb = (int)(tile / prm.nct);
             const int ct = (int)(tile - (int64_t)bb * prm.nct);
-            const int first = part * prm.chunks_per_part;
-            const int last = min(first + prm.chunks_per_part, prm.nchunks) - 1;
+            const int first = guided_start(part, prm.parts, prm.nchunks);
+            const int last = guided_start(part + 1, prm.parts, prm.nchunks) - 1;
 #pragma unroll 1
             for (int c = first; c <= last; ++c) load(u, c, bb, ct);
         };
@@ -271,9 +284,8 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
         const int64_t ch = ct * 32 + lane;
         const bool cvalid = ch < prm.HN;
         const Tin *stage = reinterpret_cast<const Tin *>(smem + s * Cfg::STAGE_BYTES);
-        const int64_t first = part * prm.chunks_per_part;  // first chunk of this unit
-        const int64_t last = (first + prm.chunks_per_part < prm.nchunks ? first + prm.chunks_per_part
-                                                                         : (int64_t)prm.nchunks) - 1;
+        const int64_t first = guided_start((int)part, prm.parts, prm.nchunks);  // first chunk of this unit
+        const int64_t last = guided_start((int)part + 1, prm.parts, prm.nchunks) - 1;
 
         // State entering chunk j -- from the previous chunk's warp, from the
         // prior at a tile's first chunk, or from the previous run of the tile
@@ -433,16 +445,6 @@ kla_forward_stream_kernel(const StreamParams prm, const __grid_constant__ FwdMap
 // inputs: 64-channel tiles, two independent recursion chains per lane).  The
 // one-channel kernel above is kept separate: compiled from this template with
 // VEC = 1 it measured 5% slower on the long fp32 workload.
-
-// Start chunk of run r of P over n chunks in the two-channel kernel, run
-// lengths in the ratio P : P-1 : ... : 1: the tickets taken last are the
-// shortest runs, so the CTAs finish closer together (1-3% faster than equal
-// runs on LM-layer shapes).  n >= P (P + 1) / 2 keeps every run non-empty
-// (the host cuts runs only for n >= 8 P).
-__device__ __forceinline__ int guided_start(int r, int P, int n) {
-    const int k = P - r;
-    return n - (int)(((int64_t)n * (k * (k + 1) / 2)) / (P * (P + 1) / 2));
-}
 
 template <typename Tin, int L, int W, int NS, int G, int VEC>
 __global__ void __launch_bounds__(32 * (W + 1), 1)
