@@ -427,7 +427,10 @@ StreamGeom stream_geom(int64_t B, int64_t T, int64_t HN, size_t esz) {
 // 2: the channel-owning streaming kernel -- its TMA geometry holds (16-byte
 //    aligned inputs and outputs, H*N*elem a multiple of 16 bytes, H*N >= 32,
 //    T >= one chunk) and there are at least 0.8 x (SM count) tiles of 32
-//    channels to keep the GPU busy, or the test hook forces it;
+//    channels to keep the GPU busy -- or at least 0.4 x (SM count) tiles of
+//    at most 16 chunks (short sequences: 64 tiles of 8-16 chunks measured
+//    5-15% faster streaming, of 32 chunks even; 16-32 tiles slower) -- or
+//    the test hook forces it;
 // 1: the chunked kernel with cross-CTA carries (any shape).
 int forward_kernel_choice(int64_t B, int64_t T, int64_t HN, size_t esz, const void *a, const void *p,
                           const void *phi, const void *b, const void *o0, const void *o1, const void *o2,
@@ -440,7 +443,9 @@ int forward_kernel_choice(int64_t B, int64_t T, int64_t HN, size_t esz, const vo
     if (!geometry) return 1;
     if (force == 2) return 2;
     const int64_t ntiles32 = B * ((HN + 31) / 32);
-    return ntiles32 * 5 >= (int64_t)sm_count() * 4 ? 2 : 1;
+    const int64_t sms = sm_count();
+    if (ntiles32 * 5 >= sms * 4) return 2;
+    return ntiles32 * 5 >= sms * 2 && (T + kSL - 1) / kSL <= 16 ? 2 : 1;
 }
 
 cudaError_t launch_clear(void *ws, size_t bytes, cudaStream_t stream) {

@@ -225,13 +225,18 @@ def test_bitwise_reproducible(kernel):
 
 def test_plan_matches_workloads():
     """On a B200 the standard workloads take the streaming kernel except the
-    tiny one (2 tiles of 32 channels cannot occupy the GPU)."""
+    tiny one (2 tiles of 32 channels cannot occupy the GPU); 64 tiles take it
+    for short sequences (at most 16 chunks) and not for longer ones."""
     kla = _kla()
     for name, expect in (("tiny", 1), ("lm_layer", 2), ("long", 2), ("stiff", 2)):
         w = wl.WORKLOADS[name]
         dt = parity.torch_dtype(w)
         z = torch.empty((w.B, w.T, w.H, w.N), dtype=dt, device=DEV)
         assert kla.forward_plan(z, z, z, z)[0] == expect, name
+        del z
+    for T, expect in ((512, (2, 1)), (1024, (1, 2))):
+        z = torch.empty((32, T, 1, 64), device=DEV)
+        assert kla.forward_plan(z, z, z, z) == expect, T
         del z
 
 
