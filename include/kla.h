@@ -201,8 +201,8 @@ kla_status_t kla_scan_forward_static(const void *a, const void *p, const void *p
 /*
  * Device workspace that kla_scan_forward_host needs (two device slots of one
  * block each, plus the scan workspace of one block), written to *bytes.
- * t_block = tokens per block, or 0 to let the library pick (about T / 16,
- * whole 64-token chunks).
+ * t_block = tokens per block, or 0 to let the library pick (about T / 64,
+ * whole 64-token chunks, at least 64 tokens).
  */
 kla_status_t kla_scan_forward_host_workspace_size(int64_t B, int64_t T, int64_t H, int64_t N,
                                                   kla_dtype_t in_dtype, int64_t t_block, size_t *bytes);
