@@ -796,7 +796,8 @@ def run_ours(args):
             "unit": UNIT, "gb_per_s": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
-                         "algorithmic_bytes_per_launch": bpt * tc_rank, "bytes_per_token_channel": bpt},
+                         "algorithmic_bytes_per_launch": bpt * tc_rank, "bytes_per_token_channel": bpt,
+                         "traffic": traffic},
             "kernel": kernel_name, "launches_per_call": plan[1],
             "timing": "the headline's timed steps: median of per-launch CUDA events, back to back "
                       "(inputs of 4.3 GB, larger than L2)"}
